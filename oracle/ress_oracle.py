@@ -1,0 +1,279 @@
+"""CPU oracle for block-sparse global attention: pooled block selection,
+block-sparse attention and per-dropped-block drift.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module.  The CUDA library
+never calls it and shares no code with it; the two meet only through the
+seeded inputs of ``block_sparse_global_mean_b200.workloads``.
+
+Everything is plain numpy in float64, written step by step in the order the
+definition gives, with no blocking, fusion or reordering.  A matmul, a sort
+and ``exp``/``log`` are the only library primitives used.
+
+Sources (the pages carry no equations; the operations are the ones the pages
+name, made exact as stated per function):
+
+* ReSS: Residual-Restoring Sparse Attention for 3D Vision Transformers
+  (thelatestinai.com), Abstract, Fig. 1, Fig. 3, Fig. 9, Table 1, Table S5,
+  Table S6.
+* VASC: Value-Aware Sparse Attention with Cross-Layer Memory
+  (paperlayer.ai), sections 4.1, 4.2, A.1, A.2, A.3.
+
+Readings taken where the pages are silent (each is repeated at its function):
+
+* the pooled score is softmax over all nb key blocks of (Qbar . Kbar) / sqrt(d),
+  d the head dimension;
+* the value contrast is the L2 norm of Vbar_j - Vbar_{j-1} with the global
+  predecessor j-1 (crossing view boundaries) and c_0 = 0, added to the
+  probability with weight lambda;
+* top-k keeps the k largest scores, ties to the lower block index, and lists
+  the kept blocks in ascending order;
+* attention is bidirectional (no causal mask) and normalised over the kept
+  tokens only; lse is the natural-log sum of exp over the kept logits;
+* the drift contribution of a dropped block uses the kept-set normaliser lse;
+  its norm is the Frobenius norm over the block's B x d contribution matrix, and
+  the drop-set drift J is the Frobenius norm of the summed contributions.
+
+Every function here is pinned by the tests in ``tests/test_oracle_pins.py``
+against closed forms, brute force, invariants or independent library routines.
+The numeric tolerances of the drift comparison (not its values) are not fixed
+by the pages.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import Iterable, Optional, Sequence, Tuple
+
+import numpy as np
+
+
+def _f64(x) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Stage 1: selection
+# ---------------------------------------------------------------------------
+
+def pool_blocks(x, block: int) -> np.ndarray:
+    """Mean of each run of ``block`` consecutive tokens, per head.
+
+    ``x`` is ``[N, H, d]``; returns ``[H, nb, d]`` with
+    out[h, i] = (1/B) * sum_{t = iB}^{iB+B-1} x[t, h].
+
+    The pooled query/key inner products of SparseVGGT are the selection basis
+    (ReSS, Table S5, SpargeAttn row); VASC pools queries, keys and values per
+    native block (VASC, sections 4.1 and A.1).
+    """
+    x = _f64(x)
+    n, h, d = x.shape
+    assert n % block == 0, "N must be a multiple of the block size"
+    nb = n // block
+    sums = x.reshape(nb, block, h, d).sum(axis=1)          # [nb, H, d]
+    return np.ascontiguousarray((sums / block).transpose(1, 0, 2))
+
+
+def block_logits(qbar, kbar) -> np.ndarray:
+    """Pooled logits s[h, i, j] = (Qbar[h, i] . Kbar[h, j]) / sqrt(d).
+
+    Reading: the temperature is sqrt(d) with d the head dimension, the usual
+    attention scale, applied to the pooled vectors.
+    """
+    qbar = _f64(qbar)
+    kbar = _f64(kbar)
+    d = qbar.shape[-1]
+    return np.matmul(qbar, kbar.transpose(0, 2, 1)) / math.sqrt(d)
+
+
+def block_probs(logits) -> np.ndarray:
+    """Softmax over all nb key blocks of each (head, query block) row."""
+    s = _f64(logits)
+    m = s.max(axis=-1, keepdims=True)
+    e = np.exp(s - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def value_contrast(vbar) -> np.ndarray:
+    """c[h, j] = || Vbar[h, j] - Vbar[h, j-1] ||_2 for j >= 1 and c[h, 0] = 0.
+
+    VASC measures the contrast between neighbouring pooled value blocks
+    (VASC, sections 4.1 and A.3).  Reading: the plain L2 norm with the global
+    predecessor j-1, and zero contrast for the first block, which has no
+    predecessor (VASC A.3 gives an unpaired block zero contrast).
+    """
+    vbar = _f64(vbar)
+    h, nb, _ = vbar.shape
+    c = np.zeros((h, nb), dtype=np.float64)
+    if nb > 1:
+        diff = vbar[:, 1:, :] - vbar[:, :-1, :]
+        c[:, 1:] = np.sqrt((diff * diff).sum(axis=-1))
+    return c
+
+
+def selection_scores(q, k, v, block: int, lam: float):
+    """The ranked quantity of the selection and its parts.
+
+    Returns a dict with ``logits`` [H, nb, nb], ``probs`` [H, nb, nb],
+    ``contrast`` [H, nb] (zeros when lam == 0) and ``score`` [H, nb, nb] =
+    probs + lam * contrast[h, None, j].
+
+    Reading: the contrast term is added to the probability (VASC section 4.1
+    says the contrast modulates the relevance; the additive form is taken).
+    """
+    qbar = pool_blocks(q, block)
+    kbar = pool_blocks(k, block)
+    logits = block_logits(qbar, kbar)
+    probs = block_probs(logits)
+    if lam != 0.0:
+        assert v is not None, "the value contrast needs V"
+        contrast = value_contrast(pool_blocks(v, block))
+    else:
+        contrast = np.zeros(probs.shape[:2], dtype=np.float64)
+    score = probs + lam * contrast[:, None, :]
+    return {"logits": logits, "probs": probs, "contrast": contrast, "score": score}
+
+
+def topk_lowest_index(score, budget: int) -> np.ndarray:
+    """Indices of the ``budget`` largest entries of each row, ascending.
+
+    A binary Top-K mask with exact capacity (VASC, section A.2): every row keeps
+    exactly ``budget`` blocks.  Ties go to the lower block index: a stable sort
+    on the negated score keeps equal scores in index order.
+    """
+    score = _f64(score)
+    order = np.argsort(-score, axis=-1, kind="stable")[..., :budget]
+    return np.sort(order, axis=-1).astype(np.int32)
+
+
+def select_blocks(q, k, v, block: int, budget: int, lam: float = 0.0,
+                  return_scores: bool = False):
+    """Stage 1 end to end: idx [H, nb, budget] int32, ascending per row."""
+    sc = selection_scores(q, k, v, block, lam)
+    idx = topk_lowest_index(sc["score"], budget)
+    if return_scores:
+        return idx, sc
+    return idx
+
+
+# ---------------------------------------------------------------------------
+# Stage 2: block-sparse attention
+# ---------------------------------------------------------------------------
+
+def _block_tokens(x_h: np.ndarray, blocks: Sequence[int], block: int) -> np.ndarray:
+    return np.concatenate([x_h[j * block:(j + 1) * block] for j in blocks], axis=0)
+
+
+def sparse_attention_block(q, k, v, kept: Sequence[int], h: int, i: int,
+                           block: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Attention output and lse of query block ``i`` of head ``h``.
+
+    For each query token n of the block: softmax over the tokens of the kept
+    key blocks only of (Q[n] . K[t]) / sqrt(d), weighted sum of V[t]; no causal
+    mask (ReSS, Table S5: global attention is bidirectional).  The kept blocks
+    are executed exactly (VASC, section 4.2: the mask is passed to the sparse
+    kernel).  lse[n] = ln sum_t exp(logit[n, t]) over the kept tokens.
+    Returns (O [B, d], lse [B]).
+    """
+    q_blk = _f64(q[i * block:(i + 1) * block, h, :])
+    k_h = _f64(k[:, h, :])
+    v_h = _f64(v[:, h, :])
+    d = q_blk.shape[-1]
+    keys = _block_tokens(k_h, kept, block)
+    vals = _block_tokens(v_h, kept, block)
+    s = (q_blk @ keys.T) / math.sqrt(d)
+    m = s.max(axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = e.sum(axis=1, keepdims=True)
+    out = (e @ vals) / l
+    lse = m[:, 0] + np.log(l[:, 0])
+    return out, lse
+
+
+def sparse_attention(q, k, v, idx, block: int,
+                     rows: Optional[Iterable[Tuple[int, int]]] = None):
+    """Stage 2 over every (head, query block) row, or over ``rows`` only.
+
+    Returns (O [N, H, d], lse [H, N]) in float64; rows not computed are NaN.
+    """
+    n, h_count, d = q.shape
+    nb = n // block
+    out = np.full((n, h_count, d), np.nan)
+    lse = np.full((h_count, n), np.nan)
+    if rows is None:
+        rows = [(h, i) for h in range(h_count) for i in range(nb)]
+    for h, i in rows:
+        o_blk, lse_blk = sparse_attention_block(q, k, v, idx[h, i], h, i, block)
+        out[i * block:(i + 1) * block, h, :] = o_blk
+        lse[h, i * block:(i + 1) * block] = lse_blk
+    return out, lse
+
+
+# ---------------------------------------------------------------------------
+# Stage 3: drift of the dropped blocks
+# ---------------------------------------------------------------------------
+
+def dropped_blocks(kept: Sequence[int], nb: int) -> np.ndarray:
+    """Complement of the kept set, ascending."""
+    mask = np.ones(nb, dtype=bool)
+    mask[np.asarray(kept, dtype=np.int64)] = False
+    return np.nonzero(mask)[0]
+
+
+def drift_block(q, k, v, kept: Sequence[int], lse_blk, h: int, i: int,
+                block: int) -> Tuple[np.ndarray, float]:
+    """Per-dropped-block drift and drop-set drift J of query block ``i``, head ``h``.
+
+    Masking a key block shifts what attention writes into the residual stream
+    (ReSS, Fig. 1 and Fig. 3(a)); the drift score measures that shift per block
+    (ReSS, Fig. 3(b)), and the drift of a drop set depends on the directions of
+    the contributions, not only their sizes (ReSS, Abstract), so the set drift
+    is the norm of their sum (ReSS, Fig. 9 plots quality against it).
+
+    For a dropped block j and query token n of block i:
+        C_j[n, :] = sum_{t in block j} exp(logit[n, t] - lse[n]) * V[t, :]
+    with lse the kept-set normaliser of stage 2 (reading: the sparse pass's
+    lse).  drift_j = ||C_j||_F over the B x d matrix, and
+    J = || sum_{j dropped} C_j ||_F.
+    Returns (drift over the dropped blocks in ascending j, J).
+    """
+    q_blk = _f64(q[i * block:(i + 1) * block, h, :])
+    k_h = _f64(k[:, h, :])
+    v_h = _f64(v[:, h, :])
+    n, d = k_h.shape
+    nb = n // block
+    lse_blk = _f64(lse_blk)
+    drop = dropped_blocks(kept, nb)
+    nd = drop.shape[0]
+    if nd == 0:
+        return np.zeros(0), 0.0
+    keys = _block_tokens(k_h, drop, block)                      # [nd*B, d]
+    vals = _block_tokens(v_h, drop, block).reshape(nd, block, d)
+    s = (q_blk @ keys.T) / math.sqrt(d)                          # [Bq, nd*B]
+    w = np.exp(s - lse_blk[:, None]).reshape(q_blk.shape[0], nd, block)
+    contrib = np.einsum("rnb,nbd->nrd", w, vals)                 # C_j: [nd, Bq, d]
+    drift = np.sqrt((contrib * contrib).sum(axis=(1, 2)))
+    total = contrib.sum(axis=0)
+    return drift, float(np.sqrt((total * total).sum()))
+
+
+def block_drift(q, k, v, idx, lse, block: int,
+                rows: Optional[Iterable[Tuple[int, int]]] = None):
+    """Stage 3 over every row, or over ``rows`` only.
+
+    Returns (drift [H, nb, nb - k], J [H, nb]) in float64; rows not computed
+    are NaN.
+    """
+    n, h_count, _ = q.shape
+    nb = n // block
+    budget = idx.shape[-1]
+    drift = np.full((h_count, nb, nb - budget), np.nan)
+    jset = np.full((h_count, nb), np.nan)
+    if rows is None:
+        rows = [(h, i) for h in range(h_count) for i in range(nb)]
+    lse = _f64(lse)
+    for h, i in rows:
+        dr, jv = drift_block(q, k, v, idx[h, i], lse[h, i * block:(i + 1) * block], h, i, block)
+        drift[h, i, :] = dr
+        jset[h, i] = jv
+    return drift, jset

@@ -1,0 +1,49 @@
+"""Write the oracle regression fixture ``oracle_tiny.json``.
+
+The pages print no worked example for this path, so the fixture is not a pin:
+it records what the oracle returns on the seeded tiny workload, so that any
+later change to the oracle's arithmetic shows up as a diff that its commit has
+to justify.  Only ``oracle/`` and the seeded input generator are called.
+
+    python tests/golden/make_golden.py
+"""
+
+import json
+import os
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, os.path.dirname(os.path.dirname(HERE)))
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import oracle  # noqa: E402
+from block_sparse_global_mean_b200 import workloads  # noqa: E402
+
+
+def main():
+    w = workloads.WORKLOADS["tiny"]
+    q, k, v = (t.to(torch.float64).numpy() for t in workloads.generate(w))
+    idx, sc = oracle.select_blocks(q, k, v, w.block, w.budget, 0.0, return_scores=True)
+    out, lse = oracle.sparse_attention(q, k, v, idx, w.block)
+    drift, jset = oracle.block_drift(q, k, v, idx, lse, w.block)
+    rows = [0, 63, 64, 300, 511]
+    fixture = {
+        "workload": "tiny",
+        "source": "oracle/ress_oracle.py on workloads.generate(WORKLOADS['tiny'])",
+        "idx": idx.tolist(),
+        "logits_row_h0_i0": sc["logits"][0, 0].tolist(),
+        "out_rows": rows,
+        "out_h1": out[rows, 1, :].tolist(),
+        "lse_h0": lse[0, rows].tolist(),
+        "drift_h0_i0": drift[0, 0].tolist(),
+        "J": jset.tolist(),
+    }
+    with open(os.path.join(HERE, "oracle_tiny.json"), "w") as f:
+        json.dump(fixture, f, indent=1)
+        f.write("\n")
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,72 @@
+"""Plant plausible mistakes in a private copy of the oracle (on the CPU) and
+check that the pins in ``test_oracle_pins`` catch every one of them."""
+
+import inspect
+import types
+
+import pytest
+
+import oracle.ress_oracle as ress_oracle
+import tests.test_oracle_pins as pins
+
+MUTATIONS = {
+    "block sum instead of block mean":
+        ("return np.ascontiguousarray((sums / block).transpose(1, 0, 2))",
+         "return np.ascontiguousarray((sums).transpose(1, 0, 2))"),
+    "temperature sqrt(8) regardless of d":
+        ("return np.matmul(qbar, kbar.transpose(0, 2, 1)) / math.sqrt(d)",
+         "return np.matmul(qbar, kbar.transpose(0, 2, 1)) / math.sqrt(8)"),
+    "contrast against the next block":
+        ("c[:, 1:] = np.sqrt((diff * diff).sum(axis=-1))",
+         "c[:, :-1] = np.sqrt((diff * diff).sum(axis=-1))"),
+    "ties to the higher index":
+        ('order = np.argsort(-score, axis=-1, kind="stable")[..., :budget]',
+         'order = (score.shape[-1] - 1 - np.argsort(-score[..., ::-1], axis=-1, kind="stable"))[..., :budget]'),
+    "contrast as a factor":
+        ("score = probs + lam * contrast[:, None, :]",
+         "score = probs * (1 + lam * contrast[:, None, :])"),
+    "lse without the row max":
+        ("lse = m[:, 0] + np.log(l[:, 0])", "lse = np.log(l[:, 0])"),
+    "drift with a shifted normaliser":
+        ("w = np.exp(s - lse_blk[:, None]).reshape(q_blk.shape[0], nd, block)",
+         "w = np.exp(s - lse_blk[:, None] - 0.01).reshape(q_blk.shape[0], nd, block)"),
+    "drift as max-abs instead of Frobenius":
+        ("drift = np.sqrt((contrib * contrib).sum(axis=(1, 2)))",
+         "drift = np.abs(contrib).max(axis=(1, 2))"),
+    "set drift as the sum of magnitudes":
+        ("return drift, float(np.sqrt((total * total).sum()))",
+         "return drift, float(drift.sum())"),
+    "a causal mask over the kept tokens":
+        ("s = (q_blk @ keys.T) / math.sqrt(d)\n    m = s.max",
+         "s = (q_blk @ keys.T) / math.sqrt(d)\n    s = s + np.triu(np.full(s.shape, -np.inf), 1)\n    m = s.max"),
+}
+
+
+def _mutant(old, new):
+    src = inspect.getsource(ress_oracle)
+    assert old in src, old
+    mod = types.ModuleType("oracle_mutant")
+    exec(compile(src.replace(old, new), "oracle_mutant", "exec"), mod.__dict__)
+    return mod
+
+
+def _pin_tests():
+    return [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_pins_catch_planted_mistake(name, monkeypatch):
+    mutant = _mutant(*MUTATIONS[name])
+    monkeypatch.setattr(pins, "oracle", mutant)
+    caught = []
+    for fn in _pin_tests():
+        try:
+            fn()
+        except Exception:   # noqa: BLE001 - any failure counts as caught
+            caught.append(fn.__name__)
+    assert caught, f"no pin caught: {name}"
+
+
+def test_unmutated_oracle_passes_every_pin():
+    for fn in _pin_tests():
+        fn()

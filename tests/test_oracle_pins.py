@@ -1,0 +1,363 @@
+"""Pins of the CPU oracle against facts that do not come from the oracle itself:
+closed forms, a hand-worked example, brute force on tiny inputs, invariants and
+independent library routines (torch float64 on the CPU).
+
+Each test is chosen so that a plausible slip in the oracle (sum instead of
+mean, sqrt(B) instead of sqrt(d), j+1 instead of j-1, ties to the higher index,
+a causal or missing mask, the dense instead of the kept-set normaliser, a norm
+other than Frobenius) fails at least one of them.
+"""
+
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from block_sparse_global_mean_b200 import workloads
+
+
+def _np64(t):
+    return t.detach().to(torch.float64).cpu().numpy()
+
+
+def _tiny_inputs():
+    w = workloads.WORKLOADS["tiny"]
+    q, k, v = workloads.generate(w)
+    return w, _np64(q), _np64(k), _np64(v)
+
+
+# --------------------------------------------------------------------------
+# Pooling
+# --------------------------------------------------------------------------
+
+def test_pool_constant_blocks_pool_to_the_constant():
+    rng = np.random.default_rng(11)
+    B, nb, H, d = 16, 5, 3, 8
+    const = rng.integers(-64, 64, size=(nb, H, d)) / 8.0  # dyadic: sums are exact
+    x = np.repeat(const, B, axis=0)                       # every block constant
+    got = oracle.pool_blocks(x, B)
+    np.testing.assert_array_equal(got, const.transpose(1, 0, 2))
+
+
+def test_pool_is_invariant_to_token_order_inside_a_block():
+    rng = np.random.default_rng(12)
+    B, nb, H, d = 16, 6, 2, 8
+    x = rng.normal(size=(nb * B, H, d))
+    perm = np.concatenate([i * B + rng.permutation(B) for i in range(nb)])
+    np.testing.assert_allclose(oracle.pool_blocks(x[perm], B), oracle.pool_blocks(x, B),
+                               rtol=0, atol=1e-14)
+
+
+def test_pool_matches_torch_mean_over_contiguous_blocks():
+    rng = np.random.default_rng(13)
+    B, nb, H, d = 32, 7, 4, 64
+    x = rng.normal(size=(nb * B, H, d))
+    ref = torch.from_numpy(x).view(nb, B, H, d).mean(dim=1).permute(1, 0, 2).numpy()
+    np.testing.assert_allclose(oracle.pool_blocks(x, B), ref, rtol=1e-13, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Pooled scores
+# --------------------------------------------------------------------------
+
+def test_logit_temperature_is_sqrt_head_dim_not_sqrt_block():
+    d = 64
+    qbar = np.zeros((1, 1, d))
+    kbar = np.zeros((1, 2, d))
+    qbar[0, 0, 0] = 2.0
+    kbar[0, 0, 0] = 3.0       # dot = 6
+    kbar[0, 1, 1] = 5.0       # dot = 0
+    s = oracle.block_logits(qbar, kbar)
+    assert s[0, 0, 0] == pytest.approx(6.0 / 8.0, abs=1e-15)
+    assert s[0, 0, 1] == 0.0
+
+
+def test_probs_rows_sum_to_one_and_match_torch_softmax():
+    w, q, k, v = _tiny_inputs()
+    sc = oracle.selection_scores(q, k, v, w.block, 0.0)
+    np.testing.assert_allclose(sc["probs"].sum(-1), 1.0, rtol=0, atol=1e-12)
+    tq = torch.from_numpy(q).view(w.n_blocks, w.block, w.heads, 64).mean(1).permute(1, 0, 2)
+    tk = torch.from_numpy(k).view(w.n_blocks, w.block, w.heads, 64).mean(1).permute(1, 0, 2)
+    ref = torch.softmax(tq @ tk.transpose(1, 2) / 8.0, dim=-1).numpy()
+    np.testing.assert_allclose(sc["probs"], ref, rtol=1e-12, atol=1e-15)
+
+
+def test_lambda_zero_ranking_by_probability_equals_ranking_by_logit():
+    w, q, k, v = _tiny_inputs()
+    sc = oracle.selection_scores(q, k, v, w.block, 0.0)
+    np.testing.assert_array_equal(oracle.topk_lowest_index(sc["probs"], w.budget),
+                                  oracle.topk_lowest_index(sc["logits"], w.budget))
+
+
+def test_value_contrast_closed_form_uses_previous_block():
+    H, nb, d = 2, 9, 64
+    vbar = np.zeros((H, nb, d))
+    for j in range(nb):
+        vbar[:, j, 0] = j * j                # ||Vbar_j - Vbar_{j-1}|| = 2j - 1
+    c = oracle.value_contrast(vbar)
+    expect = np.array([0.0] + [2.0 * j - 1.0 for j in range(1, nb)])
+    np.testing.assert_allclose(c, np.broadcast_to(expect, (H, nb)), rtol=0, atol=1e-12)
+
+
+def test_value_contrast_of_constant_values_is_zero_and_lambda_zero_reduces():
+    rng = np.random.default_rng(14)
+    B, nb, H, d = 16, 6, 2, 64
+    q = rng.normal(size=(nb * B, H, d))
+    k = rng.normal(size=(nb * B, H, d))
+    v = np.broadcast_to(rng.normal(size=(1, H, d)), (nb * B, H, d)).copy()
+    sc = oracle.selection_scores(q, k, v, B, 0.7)
+    np.testing.assert_allclose(sc["contrast"], 0.0, atol=1e-14)
+    np.testing.assert_allclose(sc["score"], sc["probs"], atol=1e-14)
+
+
+def test_contrast_enters_the_score_additively_with_weight_lambda():
+    rng = np.random.default_rng(15)
+    B, nb, H, d = 16, 6, 2, 64
+    q, k, v = (rng.normal(size=(nb * B, H, d)) for _ in range(3))
+    lam = 0.37
+    sc = oracle.selection_scores(q, k, v, B, lam)
+    vb = torch.from_numpy(v).view(nb, B, H, d).mean(1).permute(1, 0, 2)
+    c = torch.zeros(H, nb, dtype=torch.float64)
+    c[:, 1:] = torch.linalg.vector_norm(vb[:, 1:] - vb[:, :-1], dim=-1)
+    np.testing.assert_allclose(sc["score"] - sc["probs"],
+                               np.broadcast_to(lam * c.numpy()[:, None, :], sc["score"].shape),
+                               rtol=1e-12, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Top-k
+# --------------------------------------------------------------------------
+
+def _brute_force_topk(row, k):
+    """Subset maximising the score sum; ties to the lexicographically smallest
+    ascending index tuple."""
+    best, best_sum = None, -math.inf
+    for comb in itertools.combinations(range(len(row)), k):   # ascending tuples, lexicographic
+        s = float(sum(row[j] for j in comb))
+        if s > best_sum:
+            best, best_sum = comb, s
+    return list(best)
+
+
+def test_topk_equals_brute_force_on_tiny():
+    w, q, k, v = _tiny_inputs()
+    idx, sc = oracle.select_blocks(q, k, v, w.block, w.budget, 0.0, return_scores=True)
+    assert idx.shape == (w.heads, w.n_blocks, w.budget)
+    for h in range(w.heads):
+        for i in range(w.n_blocks):
+            assert list(idx[h, i]) == _brute_force_topk(sc["score"][h, i], w.budget)
+
+
+def test_topk_with_many_ties_matches_brute_force():
+    rng = np.random.default_rng(16)
+    for _ in range(40):
+        row = rng.integers(0, 3, size=8).astype(np.float64)     # heavy ties
+        for kk in (1, 3, 4, 7):
+            got = oracle.topk_lowest_index(row[None, None, :], kk)[0, 0]
+            assert list(got) == _brute_force_topk(row, kk)
+
+
+def test_topk_duplicated_key_block_keeps_lower_index():
+    # Block 6 is a copy of block 2, so their pooled scores are bitwise equal.
+    rng = np.random.default_rng(17)
+    B, nb, H, d = 64, 8, 1, 64
+    q = rng.normal(size=(nb * B, H, d))
+    k = rng.normal(size=(nb * B, H, d))
+    k[6 * B:7 * B] = k[2 * B:3 * B]
+    sc = oracle.selection_scores(q, k, None, B, 0.0)
+    for i in range(nb):
+        s = sc["score"][0, i]
+        assert s[2] == s[6]
+        order = np.argsort(-s, kind="stable")
+        pos = int(np.nonzero(order == 2)[0][0])
+        kk = pos + 1                  # the boundary falls between the twins
+        got = oracle.topk_lowest_index(sc["score"][:, i:i + 1], kk)[0, 0]
+        assert 2 in got and 6 not in got
+
+
+# --------------------------------------------------------------------------
+# Sparse attention
+# --------------------------------------------------------------------------
+
+def _sdpa(q, k, v, mask=None):
+    """torch SDPA in float64 on the CPU for one head: q [Nq, d], k/v [Nk, d]."""
+    tq = torch.from_numpy(q)[None, None]
+    tk = torch.from_numpy(k)[None, None]
+    tv = torch.from_numpy(v)[None, None]
+    am = None if mask is None else torch.from_numpy(mask)[None, None]
+    return F.scaled_dot_product_attention(tq, tk, tv, attn_mask=am)[0, 0].numpy()
+
+
+def test_full_budget_reproduces_dense_attention():
+    w, q, k, v = _tiny_inputs()
+    nb = w.n_blocks
+    idx = np.tile(np.arange(nb, dtype=np.int32), (w.heads, nb, 1))
+    out, lse = oracle.sparse_attention(q, k, v, idx, w.block)
+    for h in range(w.heads):
+        ref = _sdpa(q[:, h], k[:, h], v[:, h])
+        np.testing.assert_allclose(out[:, h], ref, rtol=1e-10, atol=1e-12)
+        ref_lse = torch.logsumexp(torch.from_numpy(q[:, h] @ k[:, h].T / 8.0), dim=-1).numpy()
+        np.testing.assert_allclose(lse[h], ref_lse, rtol=1e-12, atol=1e-12)
+
+
+def test_sparse_attention_equals_dense_with_minus_inf_mask():
+    w, q, k, v = _tiny_inputs()
+    rng = np.random.default_rng(18)
+    nb, B = w.n_blocks, w.block
+    idx = np.sort(np.stack([np.stack([rng.choice(nb, w.budget, replace=False)
+                                      for _ in range(nb)]) for _ in range(w.heads)]), -1)
+    idx = idx.astype(np.int32)
+    out, lse = oracle.sparse_attention(q, k, v, idx, B)
+    for h in range(w.heads):
+        mask = np.full((w.n_tokens, w.n_tokens), -np.inf)
+        for i in range(nb):
+            for j in idx[h, i]:
+                mask[i * B:(i + 1) * B, j * B:(j + 1) * B] = 0.0
+        ref = _sdpa(q[:, h], k[:, h], v[:, h], mask)
+        np.testing.assert_allclose(out[:, h], ref, rtol=1e-10, atol=1e-12)
+        logits = torch.from_numpy(q[:, h] @ k[:, h].T / 8.0 + mask)
+        np.testing.assert_allclose(lse[h], torch.logsumexp(logits, -1).numpy(), rtol=1e-12)
+
+
+def test_dropping_the_max_score_block_changes_the_output():
+    w, q, k, v = _tiny_inputs()
+    idx, sc = oracle.select_blocks(q, k, v, w.block, w.budget, 0.0, return_scores=True)
+    nb = w.n_blocks
+    for h in range(w.heads):
+        for i in range(nb):
+            row = sc["score"][h, i]
+            top = int(np.argmax(row))
+            alt = [j for j in np.argsort(-row, kind="stable") if j != top][:w.budget]
+            o1, _ = oracle.sparse_attention_block(q, k, v, idx[h, i], h, i, w.block)
+            o2, _ = oracle.sparse_attention_block(q, k, v, sorted(alt), h, i, w.block)
+            assert np.abs(o1 - o2).max() >= 1e-3
+
+
+# --------------------------------------------------------------------------
+# Hand-worked example through all three stages (d = 4, B = 2, N = 4, k = 1)
+# --------------------------------------------------------------------------
+
+def _hand_inputs():
+    q = np.zeros((4, 1, 4)); k = np.zeros((4, 1, 4)); v = np.zeros((4, 1, 4))
+    q[0, 0, 0] = 2.0          # Qbar_0 = (1, 0, 0, 0)
+    q[2, 0, 1] = 2.0          # Qbar_1 = (0, 1, 0, 0)
+    k[0, 0, 0] = 4.0          # Kbar_0 = (2, 0, 0, 0)
+    k[3, 0, 1] = 6.0          # Kbar_1 = (0, 3, 0, 0)
+    for t in range(4):
+        v[t, 0, t] = 1.0      # V_t = e_t
+    return q, k, v
+
+
+def test_hand_worked_example():
+    q, k, v = _hand_inputs()
+    e = math.e
+    sc = oracle.selection_scores(q, k, v, 2, 0.0)
+    # logits = Qbar Kbar^T / sqrt(4): [[1, 0], [0, 1.5]]
+    np.testing.assert_allclose(sc["logits"][0], [[1.0, 0.0], [0.0, 1.5]], atol=1e-15)
+    np.testing.assert_allclose(sc["probs"][0], [[e / (e + 1), 1 / (e + 1)],
+                                                [1 / (1 + e ** 1.5), e ** 1.5 / (1 + e ** 1.5)]],
+                               rtol=1e-14)
+    idx = oracle.topk_lowest_index(sc["score"], 1)
+    assert idx[0, :, 0].tolist() == [0, 1]
+    out, lse = oracle.sparse_attention(q, k, v, idx, 2)
+    # token 0: logits (4, 0) over keys 0, 1; token 1: (0, 0); token 2: (0, 6) over keys 2, 3.
+    expect = np.array([[e ** 4 / (1 + e ** 4), 1 / (1 + e ** 4), 0, 0],
+                       [0.5, 0.5, 0, 0],
+                       [0, 0, 1 / (1 + e ** 6), e ** 6 / (1 + e ** 6)],
+                       [0, 0, 0.5, 0.5]])
+    np.testing.assert_allclose(out[:, 0], expect, rtol=1e-14, atol=1e-16)
+    np.testing.assert_allclose(lse[0], [math.log(1 + e ** 4), math.log(2),
+                                        math.log(1 + e ** 6), math.log(2)], rtol=1e-14)
+    drift, jset = oracle.block_drift(q, k, v, idx, lse, 2)
+    # Query block 0 drops block 1: all four logits are 0, so
+    # C = [[0, 0, 1, 1] / (1 + e^4), [0, 0, 1, 1] / 2].
+    d0 = math.sqrt(2.0 / (1 + e ** 4) ** 2 + 2.0 / 4.0)
+    # Query block 1 drops block 0: C = [[1, 1, 0, 0] / (1 + e^6), [1, 1, 0, 0] / 2].
+    d1 = math.sqrt(2.0 / (1 + e ** 6) ** 2 + 2.0 / 4.0)
+    np.testing.assert_allclose(drift[0, :, 0], [d0, d1], rtol=1e-14)
+    np.testing.assert_allclose(jset[0], [d0, d1], rtol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# Drift
+# --------------------------------------------------------------------------
+
+def test_drift_of_an_empty_drop_set_is_zero():
+    w, q, k, v = _tiny_inputs()
+    nb = w.n_blocks
+    idx = np.tile(np.arange(nb, dtype=np.int32), (w.heads, nb, 1))
+    _, lse = oracle.sparse_attention(q, k, v, idx, w.block)
+    drift, jset = oracle.block_drift(q, k, v, idx, lse, w.block)
+    assert drift.shape == (w.heads, nb, 0)
+    np.testing.assert_array_equal(jset, 0.0)
+
+
+def test_drift_reconstructs_dense_attention():
+    """O_dense = (O_sparse + sum_j C_j) / (1 + sum_j r_j), r_j = sum_t exp(s - lse).
+
+    The expected J = ||sum_j C_j||_F is formed from torch SDPA and torch
+    logsumexp only, then compared with the oracle's J.
+    """
+    w, q, k, v = _tiny_inputs()
+    idx = oracle.select_blocks(q, k, v, w.block, w.budget)
+    _, lse = oracle.sparse_attention(q, k, v, idx, w.block)
+    _, jset = oracle.block_drift(q, k, v, idx, lse, w.block)
+    B, nb = w.block, w.n_blocks
+    for h in range(w.heads):
+        logits = q[:, h] @ k[:, h].T / 8.0
+        dense = _sdpa(q[:, h], k[:, h], v[:, h])
+        for i in range(nb):
+            keep = np.full(w.n_tokens, False)
+            for j in idx[h, i]:
+                keep[j * B:(j + 1) * B] = True
+            rows = slice(i * B, (i + 1) * B)
+            mask = np.where(keep, 0.0, -np.inf)[None, :].repeat(B, 0)
+            sparse = _sdpa(q[rows, h], k[:, h], v[:, h], mask)
+            lse_t = torch.logsumexp(torch.from_numpy(logits[rows] + mask), -1).numpy()
+            r = np.exp(logits[rows][:, ~keep] - lse_t[:, None]).sum(-1)
+            total_c = dense[rows] * (1.0 + r[:, None]) - sparse
+            assert jset[h, i] == pytest.approx(np.linalg.norm(total_c), rel=1e-9)
+
+
+def test_drift_of_one_dropped_block_equals_j_and_triangle_inequality_holds():
+    w, q, k, v = _tiny_inputs()
+    nb = w.n_blocks
+    rng = np.random.default_rng(19)
+    idx1 = np.stack([np.stack([np.sort(rng.choice(nb, nb - 1, replace=False))
+                               for _ in range(nb)]) for _ in range(w.heads)]).astype(np.int32)
+    _, lse1 = oracle.sparse_attention(q, k, v, idx1, w.block)
+    drift1, j1 = oracle.block_drift(q, k, v, idx1, lse1, w.block)
+    np.testing.assert_allclose(drift1[..., 0], j1, rtol=1e-14)
+    idx = oracle.select_blocks(q, k, v, w.block, w.budget)
+    _, lse = oracle.sparse_attention(q, k, v, idx, w.block)
+    drift, jset = oracle.block_drift(q, k, v, idx, lse, w.block)
+    assert np.all(jset <= drift.sum(-1) * (1 + 1e-12))
+    assert np.all(jset < drift.sum(-1))   # generic contributions are not parallel
+
+
+def test_drift_closed_form_with_zero_queries_and_orthogonal_values():
+    """Q = 0 makes every logit 0, so exp(s - lse) = 1 / (k B) for all tokens and
+    C_j[n] = sum_{t in j} V[t] / (k B) for every query row.  Values of dropped
+    block j live on coordinate j only, so the C_j are orthogonal and
+    J^2 = sum_j drift_j^2."""
+    B, nb, H, d, budget = 8, 6, 1, 16, 2
+    rng = np.random.default_rng(20)
+    q = np.zeros((nb * B, H, d))
+    k = rng.normal(size=(nb * B, H, d))
+    v = np.zeros((nb * B, H, d))
+    for j in range(nb):
+        v[j * B:(j + 1) * B, 0, j] = rng.normal(size=B)
+    idx = np.tile(np.array([0, 1], dtype=np.int32), (H, nb, 1))
+    _, lse = oracle.sparse_attention(q, k, v, idx, B)
+    np.testing.assert_allclose(lse, math.log(budget * B), rtol=1e-14)
+    drift, jset = oracle.block_drift(q, k, v, idx, lse, B)
+    for i in range(nb):
+        for r, j in enumerate(range(2, nb)):
+            col_sum = v[j * B:(j + 1) * B, 0, j].sum()
+            expect = math.sqrt(B) * abs(col_sum) / (budget * B)
+            assert drift[0, i, r] == pytest.approx(expect, rel=1e-12)
+        assert jset[0, i] == pytest.approx(math.sqrt((drift[0, i] ** 2).sum()), rel=1e-12)
