@@ -1,0 +1,534 @@
+// Stage 3: per-dropped-block drift on tcgen05 tensor cores.
+//
+// For a 128-row query tile (two 64-token query blocks, or one 128-token block)
+// the CTA visits the union of the tile's dropped key blocks in ascending order.
+// Per 128-key chunk:
+//   S = Q K^T                          (M=128, N=128, K=64) into TMEM
+//   P = exp(S / 8 - lse)  as bf16     (softmax warps; the kept-set lse of the
+//                                      sparse pass; 0 where the row keeps the block)
+//   C_j = P[:, block j] V[block j]    (one fresh TMEM accumulator per dropped block)
+//   T  += P V                         (running sum of every C_j of the row)
+// and the softmax warps reduce ||C_j||_F over the block's rows, writing
+// drift[h][i][r] (r = rank of j among the dropped blocks of query block i);
+// at the end set_drift[h][i] = ||T||_F.
+//
+// Source: ReSS (thelatestinai.com) Abstract, Fig. 1 and Fig. 3: masking a block
+// shifts what attention writes into the residual stream; the drift score
+// measures that shift per block, and the drift of a drop set depends on the
+// directions of the contributions, so the set drift is the norm of their sum.
+//
+// Warp roles as in the attention kernel (warp 0 TMA, warp 1 TMEM + MMA,
+// warps 2-5 exponentials and reductions); one CTA per SM (512 TMEM columns).
+#include "ress_common.cuh"
+#include "ress_internal.h"
+
+namespace ress {
+
+namespace {
+
+constexpr int kRows = 128;
+constexpr int kStages = 2;
+constexpr int kThreads = 192;
+constexpr uint32_t kQBytes = 128 * 128;
+constexpr uint32_t kSubBytes = 64 * 128;
+constexpr uint32_t kStageBytes = 4 * kSubBytes;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;     // S (fp32) / P (bf16, cols 0..63)
+constexpr uint32_t kColC0 = 128;  // contribution of sub-block 0 (or the whole 128-key block)
+constexpr uint32_t kColC1 = 192;  // contribution of sub-block 1 (block 64 only)
+constexpr uint32_t kColT = 256;   // running sum of the contributions
+
+struct DriftParams {
+  DeviceError* err;
+  int n;
+  int heads;
+  int nb;
+  int block;
+  int budget;
+  int tiles_per_head;
+  const int32_t* idx;
+  const float* lse;
+  float* drift;
+  float* set_drift;
+};
+
+struct __align__(8) Ctl {
+  uint64_t q_full;
+  uint64_t kv_full[kStages];
+  uint64_t kv_empty[kStages];
+  uint64_t s_full;
+  uint64_t p_full;
+  uint64_t c_full;
+  uint64_t c_free;
+  uint64_t t_full;
+  uint64_t mma_done;
+  uint64_t red_full;    // the four softmax warps posted this chunk's partial sums
+  uint64_t tred_full;   // ... and their partial sums of the running total
+  uint32_t tmem_base;
+  int abort_flag;
+  int n_entries;
+  int pad;
+  float partial[2][4][2];   // [chunk parity][quad][sub-block] sums of squares
+  float tpartial[4];
+};
+
+__host__ __device__ inline int words_for(int nb) { return (nb + 31) >> 5; }
+
+size_t drift_smem_bytes(int nb) {
+  return 1024 + kQBytes + kStages * kStageBytes + sizeof(Ctl) +
+         sizeof(uint32_t) * (4 * (size_t)words_for(nb) + (size_t)nb);
+}
+
+__device__ __forceinline__ void chunk_info(const uint32_t* list, int n_entries, int block, int c,
+                                           int& t0, int& t1, uint32_t& j0, uint32_t& j1,
+                                           uint32_t& m0, uint32_t& m1) {
+  if (block == 64) {
+    const uint32_t e0 = list[2 * c];
+    j0 = e0 & 0x3FFFFFFFu;
+    t0 = (int)j0 * 64;
+    m0 = e0 >> 30;
+    if (2 * c + 1 < n_entries) {
+      const uint32_t e1 = list[2 * c + 1];
+      j1 = e1 & 0x3FFFFFFFu;
+      t1 = (int)j1 * 64;
+      m1 = e1 >> 30;
+    } else {
+      j1 = j0;
+      t1 = t0;
+      m1 = 0;
+    }
+  } else {
+    const uint32_t e0 = list[c];
+    j0 = j1 = e0 & 0x3FFFFFFFu;
+    t0 = (int)j0 * 128;
+    t1 = t0 + 64;
+    m0 = m1 = 3u;
+  }
+}
+
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          DeviceError* err, int detail) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, err, detail);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Rank of block j among the blocks NOT set in `kept` (bitmap) below j.
+__device__ __forceinline__ int dropped_rank(const uint32_t* kept, const uint32_t* prefix, int j) {
+  const uint32_t below = kept[j >> 5] & ((1u << (j & 31)) - 1u);
+  return j - (int)(prefix[j >> 5] + __popc(below));
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    block_drift_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v, const DriftParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + kQBytes;
+  Ctl* ctl = reinterpret_cast<Ctl*>(sKV + kStages * kStageBytes);
+  const int W = words_for(p.nb);
+  uint32_t* keptA = reinterpret_cast<uint32_t*>(ctl + 1);
+  uint32_t* keptB = keptA + W;
+  uint32_t* prefA = keptB + W;
+  uint32_t* prefB = prefA + W;
+  uint32_t* list = prefB + W;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int h = blockIdx.x / p.tiles_per_head;
+  const int tile = blockIdx.x % p.tiles_per_head;
+  const int row0 = tile * kRows;
+  const int nsets = (p.block == 64) ? 2 : 1;
+  const int qb0 = (p.block == 64) ? 2 * tile : tile;
+  const bool validB = (p.block == 64) && (qb0 + 1 < p.nb);
+  const int n_drop = p.nb - p.budget;
+
+  const uint32_t bar_q = smem_addr(&ctl->q_full);
+  const uint32_t bar_s = smem_addr(&ctl->s_full);
+  const uint32_t bar_p = smem_addr(&ctl->p_full);
+  const uint32_t bar_c = smem_addr(&ctl->c_full);
+  const uint32_t bar_cf = smem_addr(&ctl->c_free);
+  const uint32_t bar_t = smem_addr(&ctl->t_full);
+  const uint32_t bar_done = smem_addr(&ctl->mma_done);
+  const uint32_t bar_red = smem_addr(&ctl->red_full);
+  const uint32_t bar_tred = smem_addr(&ctl->tred_full);
+  volatile int* abortf = &ctl->abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    mbar_init(bar_red, 128);
+    mbar_init(bar_tred, 128);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_addr(&ctl->kv_full[s]), 1);
+      mbar_init(smem_addr(&ctl->kv_empty[s]), 1);
+    }
+    mbar_init(bar_s, 1);
+    mbar_init(bar_p, 128);
+    mbar_init(bar_c, 1);
+    mbar_init(bar_cf, 128);
+    mbar_init(bar_t, 1);
+    mbar_init(bar_done, 1);
+    ctl->abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(&ctl->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  for (int w = threadIdx.x; w < 2 * W; w += kThreads) keptA[w] = 0u;
+  __syncthreads();
+
+  for (int e = threadIdx.x; e < nsets * p.budget; e += kThreads) {
+    const int s = e / p.budget;
+    const int r = e - s * p.budget;
+    const int qb = qb0 + s;
+    if (qb >= p.nb) continue;
+    const int j = p.idx[((size_t)h * p.nb + qb) * p.budget + r];
+    if (j < 0 || j >= p.nb) {
+      raise_device_error(p.err, RESS_ERR_BAD_INDEX, 2);
+      continue;
+    }
+    atomicOr(&(s ? keptB : keptA)[j >> 5], 1u << (j & 31));
+  }
+  __syncthreads();
+
+  // Prefix popcounts of the kept bitmaps and the union of the dropped sets.
+  if (warp == 0) {
+    int base = 0, baseA = 0, baseB = 0;
+    for (int w0 = 0; w0 < W; w0 += 32) {
+      const int w = w0 + lane;
+      uint32_t valid = 0u;
+      if (w < W) valid = (w == W - 1 && (p.nb & 31)) ? ((1u << (p.nb & 31)) - 1u) : 0xffffffffu;
+      const uint32_t ka = (w < W) ? keptA[w] : 0u;
+      const uint32_t kb = (w < W) ? keptB[w] : 0u;
+      const uint32_t a = ~ka & valid;
+      const uint32_t b = (nsets == 2) ? (validB ? (~kb & valid) : 0u) : a;
+      int ca = __popc(ka), cb = __popc(kb);
+      int ia = ca, ib = cb;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int ya = __shfl_up_sync(0xffffffffu, ia, o);
+        const int yb = __shfl_up_sync(0xffffffffu, ib, o);
+        if (lane >= o) {
+          ia += ya;
+          ib += yb;
+        }
+      }
+      if (w < W) {
+        prefA[w] = (uint32_t)(baseA + ia - ca);
+        prefB[w] = (uint32_t)(baseB + ib - cb);
+      }
+      baseA += __shfl_sync(0xffffffffu, ia, 31);
+      baseB += __shfl_sync(0xffffffffu, ib, 31);
+      uint32_t u = a | b;
+      const int cnt = __popc(u);
+      int incl = cnt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int pos = base + incl - cnt;
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        u &= u - 1u;
+        const uint32_t mem = ((a >> bit) & 1u) | (((b >> bit) & 1u) << 1);
+        list[pos++] = (uint32_t)(w * 32 + bit) | (mem << 30);
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) ctl->n_entries = base;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = ctl->tmem_base;
+  const int n_entries = ctl->n_entries;
+  const int n_chunks = (p.block == 64) ? (n_entries + 1) / 2 : n_entries;
+
+  if (warp == 0) {
+    if (lane == 0 && n_chunks > 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(bar_q, kQBytes);
+      tma_load_3d(smem_addr(sQ), &tm_q, bar_q, 0, h, row0);
+      int issued = 0;
+      for (int c = 0; c < n_chunks; ++c) {
+        const int s = c % kStages;
+        if (c >= kStages &&
+            !mbar_wait(smem_addr(&ctl->kv_empty[s]), ((c / kStages) - 1) & 1, abortf, p.err, 40))
+          break;
+        int t0, t1;
+        uint32_t j0, j1, m0, m1;
+        chunk_info(list, n_entries, p.block, c, t0, t1, j0, j1, m0, m1);
+        uint8_t* st = sKV + s * kStageBytes;
+        const uint32_t bar = smem_addr(&ctl->kv_full[s]);
+        mbar_arrive_expect_tx(bar, kStageBytes);
+        tma_load_3d(smem_addr(st), &tm_k, bar, 0, h, t0);
+        tma_load_3d(smem_addr(st + kSubBytes), &tm_k, bar, 0, h, t1);
+        tma_load_3d(smem_addr(st + 2 * kSubBytes), &tm_v, bar, 0, h, t0);
+        tma_load_3d(smem_addr(st + 3 * kSubBytes), &tm_v, bar, 0, h, t1);
+        issued = c + 1;
+      }
+      for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c)
+        mbar_wait_drain(smem_addr(&ctl->kv_full[c % kStages]), (c / kStages) & 1, p.err, 41);
+      mbar_wait_drain(bar_q, 0, p.err, 42);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && n_chunks > 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, 128, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(128, 64, true);
+      const uint32_t tS = tmem + kColS;
+      const uint64_t dq = smem_desc_sw128(smem_addr(sQ), 16, 1024);
+      bool ok = mbar_wait(bar_q, 0, abortf, p.err, 50);
+      for (int c = 0; ok && c < n_chunks; ++c) {
+        const int s = c % kStages;
+        if (!mbar_wait(smem_addr(&ctl->kv_full[s]), (c / kStages) & 1, abortf, p.err, 51)) break;
+        tc_fence_after();
+        const uint64_t dk = smem_desc_sw128(smem_addr(sKV + s * kStageBytes), 16, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tS, dq + (uint64_t)(kk * 2), dk + (uint64_t)(kk * 2), idS, kk > 0 ? 1u : 0u);
+        mma_commit(bar_s);
+        if (!mbar_wait(bar_p, c & 1, abortf, p.err, 52)) break;
+        if (c > 0 && !mbar_wait(bar_cf, (c - 1) & 1, abortf, p.err, 53)) break;
+        tc_fence_after();
+        const uint32_t vaddr = smem_addr(sKV + s * kStageBytes + 2 * kSubBytes);
+        if (p.block == 64) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            mma_ts(tmem + kColC0, tS + kk * 8,
+                   smem_desc_sw128(vaddr + kk * 2048, 16384, 1024), idPV, kk > 0 ? 1u : 0u);
+            mma_ts(tmem + kColC1, tS + 32 + kk * 8,
+                   smem_desc_sw128(vaddr + kSubBytes + kk * 2048, 16384, 1024), idPV,
+                   kk > 0 ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + kColC0, tS + kk * 8, smem_desc_sw128(vaddr + kk * 2048, 16384, 1024),
+                   idPV, kk > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + kColT, tS + kk * 8, smem_desc_sw128(vaddr + kk * 2048, 16384, 1024), idPV,
+                 (c > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(bar_c);
+        mma_commit(smem_addr(&ctl->kv_empty[s]));
+        if (c == n_chunks - 1) mma_commit(bar_t);
+      }
+      mma_commit(bar_done);
+      mbar_wait_drain(bar_done, 0, p.err, 54);
+    }
+    __syncwarp();
+  } else {
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    const int half = row >> 6;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + kColS + lane_off;
+    const float kScaleLog2 = 1.4426950408889634f * 0.125f;
+    const int tok = row0 + row;
+    const float lse2 = (tok < p.n) ? p.lse[(size_t)h * p.n + tok] * 1.4426950408889634f : 0.f;
+    const float neg_l = -lse2;
+    const int sub_tid = threadIdx.x - 64;   // 0..127 among the softmax warps
+    bool ok = true;
+    for (int c = 0; c < n_chunks; ++c) {
+      if (!warp_wait(bar_s, c & 1, abortf, p.err, 60)) { ok = false; break; }
+      tc_fence_after();
+      int t0, t1;
+      uint32_t j0, j1, m0, m1;
+      chunk_info(list, n_entries, p.block, c, t0, t1, j0, j1, m0, m1);
+      const bool use0 = (m0 >> half) & 1u;
+      const bool use1 = (m1 >> half) & 1u;
+      if (use0 || use1) {
+        uint32_t r[4][32];
+        tmem_ld32(tS, r[0]);
+        tmem_ld32(tS + 32, r[1]);
+        tmem_ld32(tS + 64, r[2]);
+        tmem_ld32(tS + 96, r[3]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const bool use = (g < 2) ? use0 : use1;
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e]), kScaleLog2, neg_l));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e + 1]), kScaleLog2, neg_l));
+            pk[e] = use ? pack_bf16x2(p0, p1) : 0u;
+          }
+          tmem_st16(tS + 16 * g, pk);
+        }
+      } else {
+        uint32_t z[32];
+#pragma unroll
+        for (int u = 0; u < 32; ++u) z[u] = 0u;
+        tmem_st32(tS, z);
+        tmem_st32(tS + 32, z);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_p);
+
+      if (!warp_wait(bar_c, c & 1, abortf, p.err, 61)) { ok = false; break; }
+      tc_fence_after();
+      float ss0 = 0.f, ss1 = 0.f;
+      {
+        uint32_t cv[32];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          tmem_ld32(tmem + kColC0 + lane_off + 32 * g, cv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const float x = __uint_as_float(cv[u]);
+            ss0 = fmaf(x, x, ss0);
+          }
+        }
+        if (p.block == 64) {
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            tmem_ld32(tmem + kColC1 + lane_off + 32 * g, cv);
+            tmem_ld_wait();
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+              const float x = __uint_as_float(cv[u]);
+              ss1 = fmaf(x, x, ss1);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_cf);
+      ss0 = warp_sum(ss0);
+      ss1 = warp_sum(ss1);
+      if (lane == 0) {
+        ctl->partial[c & 1][quad][0] = ss0;
+        ctl->partial[c & 1][quad][1] = ss1;
+      }
+      __syncwarp();
+      mbar_arrive(bar_red);
+      // Writers: sub_tid 0..3 -> (half, sub-block) for block 64; sub_tid 0 for
+      // block 128.  A slot is rewritten two chunks later at the earliest, and
+      // no warp can run two chunks ahead of the writers (every chunk's PV
+      // waits for all 128 softmax threads).
+      const bool writer = (p.block == 64) ? (sub_tid < 4) : (sub_tid == 0);
+      const bool have = writer && mbar_wait(bar_red, c & 1, abortf, p.err, 63);
+      if (!have) {
+        // not a writer (or the wait gave up)
+      } else if (p.block == 64) {
+        {
+          const int hf = sub_tid >> 1, sb = sub_tid & 1;
+          const uint32_t mem = sb ? m1 : m0;
+          const int qb = qb0 + hf;
+          if (((mem >> hf) & 1u) && qb < p.nb) {
+            const int j = (int)(sb ? j1 : j0);
+            const float ss = ctl->partial[c & 1][2 * hf][sb] + ctl->partial[c & 1][2 * hf + 1][sb];
+            const int rnk = dropped_rank(hf ? keptB : keptA, hf ? prefB : prefA, j);
+            if (rnk >= 0 && rnk < n_drop)
+              p.drift[((size_t)h * p.nb + qb) * n_drop + rnk] = sqrtf(ss);
+            else
+              raise_device_error(p.err, RESS_ERR_BAD_INDEX, 3);
+          }
+        }
+      } else if (sub_tid == 0) {
+        const float ss = ctl->partial[c & 1][0][0] + ctl->partial[c & 1][1][0] +
+                         ctl->partial[c & 1][2][0] + ctl->partial[c & 1][3][0];
+        const int rnk = dropped_rank(keptA, prefA, (int)j0);
+        if (rnk >= 0 && rnk < n_drop)
+          p.drift[((size_t)h * p.nb + qb0) * n_drop + rnk] = sqrtf(ss);
+        else
+          raise_device_error(p.err, RESS_ERR_BAD_INDEX, 3);
+      }
+      __syncwarp();
+    }
+    // Drop-set drift J = ||sum_j C_j||_F.
+    float tss = 0.f;
+    if (ok && n_chunks > 0) {
+      if (warp_wait(bar_t, 0, abortf, p.err, 62)) {
+        tc_fence_after();
+        uint32_t tv[32];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          tmem_ld32(tmem + kColT + lane_off + 32 * g, tv);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) {
+            const float x = __uint_as_float(tv[u]);
+            tss = fmaf(x, x, tss);
+          }
+        }
+      }
+    }
+    tss = warp_sum(tss);
+    if (lane == 0) ctl->tpartial[quad] = tss;
+    __syncwarp();
+    mbar_arrive(bar_tred);
+    const bool twriter = (p.block == 64) ? (sub_tid < 2) : (sub_tid == 0);
+    if (p.set_drift && twriter && mbar_wait(bar_tred, 0, abortf, p.err, 64)) {
+      if (p.block == 64) {
+        if (sub_tid < 2) {
+          const int qb = qb0 + sub_tid;
+          if (qb < p.nb)
+            p.set_drift[(size_t)h * p.nb + qb] =
+                sqrtf(ctl->tpartial[2 * sub_tid] + ctl->tpartial[2 * sub_tid + 1]);
+        }
+      } else if (sub_tid == 0) {
+        p.set_drift[(size_t)h * p.nb + qb0] = sqrtf(ctl->tpartial[0] + ctl->tpartial[1] +
+                                                    ctl->tpartial[2] + ctl->tpartial[3]);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
+
+ress_status launch_drift(const Geometry& g, const void* q, const void* k, const void* v,
+                         int budget, const int32_t* idx, const float* lse, float* drift,
+                         float* set_drift, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  if (!make_token_map(&tq, q, g, 128) || !make_token_map(&tk, k, g, 64) ||
+      !make_token_map(&tv, v, g, 64))
+    return RESS_ERR_CUDA;
+  DriftParams p{};
+  p.err = device_error_ptr();
+  if (p.err == nullptr) return RESS_ERR_CUDA;
+  p.n = (int)g.n;
+  p.heads = g.heads;
+  p.nb = g.nb;
+  p.block = g.block;
+  p.budget = budget;
+  p.tiles_per_head = (g.block == 64) ? (g.nb + 1) / 2 : g.nb;
+  p.idx = idx;
+  p.lse = lse;
+  p.drift = drift;
+  p.set_drift = set_drift;
+  const size_t smem = drift_smem_bytes(g.nb);
+  if (cudaFuncSetAttribute(block_drift_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return RESS_ERR_CUDA;
+  block_drift_kernel<<<(unsigned)(g.heads * p.tiles_per_head), kThreads, smem, st>>>(tq, tk, tv,
+                                                                                     p);
+  return cudaGetLastError() == cudaSuccess ? RESS_OK : RESS_ERR_CUDA;
+}
+
+}  // namespace ress

@@ -1,0 +1,208 @@
+"""Python binding of the C ABI in ``include/ress.h`` (ctypes).
+
+Argument marshalling only: every step of the path runs in the CUDA kernels of
+``libress.so``.  PyTorch supplies device memory and the current stream.  If
+the library is missing, importing this module raises ImportError; there is no
+fallback implementation.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG_DIR, "libress.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m block_sparse_global_mean_b200.build` "
+        "(this package has no CPU fallback)")
+
+lib = ctypes.CDLL(LIB_PATH)
+
+RESS_OK = 0
+RESS_ERR_INVALID_ARG = 1
+RESS_ERR_UNSUPPORTED = 2
+RESS_ERR_WORKSPACE = 3
+RESS_ERR_CUDA = 4
+RESS_ERR_TIMEOUT = 5
+RESS_ERR_BAD_INDEX = 6
+
+RESS_BF16 = 0
+RESS_F32 = 1
+
+
+class ress_shape(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int64), ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("block", ctypes.c_int32), ("dtype", ctypes.c_int32)]
+
+
+_P = ctypes.c_void_p
+_SHAPE = ctypes.POINTER(ress_shape)
+
+lib.ress_version.restype = ctypes.c_int
+lib.ress_version.argtypes = []
+lib.ress_status_string.restype = ctypes.c_char_p
+lib.ress_status_string.argtypes = [ctypes.c_int]
+lib.ress_select_workspace_bytes.restype = ctypes.c_size_t
+lib.ress_select_workspace_bytes.argtypes = [_SHAPE, ctypes.c_float]
+lib.ress_select_blocks.restype = ctypes.c_int
+lib.ress_select_blocks.argtypes = [_SHAPE, _P, _P, _P, ctypes.c_int32, ctypes.c_float, _P, _P,
+                                   ctypes.c_size_t, _P]
+lib.ress_attn_workspace_bytes.restype = ctypes.c_size_t
+lib.ress_attn_workspace_bytes.argtypes = [_SHAPE]
+lib.ress_block_sparse_attn.restype = ctypes.c_int
+lib.ress_block_sparse_attn.argtypes = [_SHAPE, _P, _P, _P, ctypes.c_int32, _P, _P, ctypes.c_int32,
+                                       _P, _P, ctypes.c_size_t, _P]
+lib.ress_block_drift.restype = ctypes.c_int
+lib.ress_block_drift.argtypes = [_SHAPE, _P, _P, _P, ctypes.c_int32, _P, _P, _P, _P, _P,
+                                 ctypes.c_size_t, _P]
+lib.ress_check_device_errors.restype = ctypes.c_int
+lib.ress_check_device_errors.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
+
+
+class RessError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = lib.ress_status_string(status).decode()
+        super().__init__(f"{where}: {msg} (status {status})")
+
+
+def _check(status: int, where: str) -> None:
+    if status != RESS_OK:
+        raise RessError(status, where)
+
+
+def make_shape(n: int, heads: int, block: int, dtype: torch.dtype, head_dim: int = 64) -> ress_shape:
+    if dtype == torch.bfloat16:
+        code = RESS_BF16
+    elif dtype == torch.float32:
+        code = RESS_F32
+    else:
+        raise TypeError(f"unsupported dtype {dtype}")
+    return ress_shape(n, heads, head_dim, block, code)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream_ptr(stream: Optional[torch.cuda.Stream], device: torch.device) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return s.cuda_stream
+
+
+def _shape_of(q: torch.Tensor, block: int) -> ress_shape:
+    if q.dim() != 3:
+        raise ValueError("q, k, v must be [N, H, d]")
+    n, h, d = q.shape
+    return make_shape(n, h, block, q.dtype, d)
+
+
+def select_workspace_bytes(n: int, heads: int, block: int, dtype: torch.dtype, lam: float) -> int:
+    sh = make_shape(n, heads, block, dtype)
+    return int(lib.ress_select_workspace_bytes(ctypes.byref(sh), ctypes.c_float(lam)))
+
+
+def attn_workspace_bytes(n: int, heads: int, block: int, dtype: torch.dtype) -> int:
+    sh = make_shape(n, heads, block, dtype)
+    return int(lib.ress_attn_workspace_bytes(ctypes.byref(sh)))
+
+
+def ress_select_blocks(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor], budget: int,
+                       lam: float, block: int, idx: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None,
+                       stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Stage 1: returns idx [H, nb, budget] int32 (ascending kept blocks per row)."""
+    sh = _shape_of(q, block)
+    n, h = q.shape[0], q.shape[1]
+    nb = n // block
+    if idx is None:
+        idx = torch.empty((h, nb, budget), dtype=torch.int32, device=q.device)
+    need = int(lib.ress_select_workspace_bytes(ctypes.byref(sh), ctypes.c_float(lam)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    status = lib.ress_select_blocks(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(budget),
+                                    ctypes.c_float(lam), _ptr(idx), _ptr(workspace),
+                                    workspace.numel(), _stream_ptr(stream, q.device))
+    _check(status, "ress_select_blocks")
+    return idx
+
+
+def ress_block_sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor,
+                           block: int, out: Optional[torch.Tensor] = None,
+                           lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+                           workspace: Optional[torch.Tensor] = None,
+                           stream: Optional[torch.cuda.Stream] = None,
+                           out_dtype: Optional[torch.dtype] = None
+                           ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Stage 2: returns (out [N, H, 64], lse [H, N] float32 or None).
+
+    The output dtype is ``out.dtype`` if ``out`` is given, else ``out_dtype``,
+    else the input dtype."""
+    sh = _shape_of(q, block)
+    n, h = q.shape[0], q.shape[1]
+    budget = idx.shape[-1]
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    out_code = RESS_F32 if out.dtype == torch.float32 else (
+        RESS_BF16 if out.dtype == torch.bfloat16 else None)
+    if out_code is None:
+        raise TypeError(f"unsupported output dtype {out.dtype}")
+    if lse is None and want_lse:
+        lse = torch.empty((h, n), dtype=torch.float32, device=q.device)
+    need = int(lib.ress_attn_workspace_bytes(ctypes.byref(sh)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    status = lib.ress_block_sparse_attn(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(budget),
+                                        _ptr(idx), _ptr(out), out_code, _ptr(lse), _ptr(workspace),
+                                        0 if workspace is None else workspace.numel(),
+                                        _stream_ptr(stream, q.device))
+    _check(status, "ress_block_sparse_attn")
+    return out, lse
+
+
+def ress_block_drift(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor,
+                     lse: torch.Tensor, block: int, drift: Optional[torch.Tensor] = None,
+                     set_drift: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None,
+                     stream: Optional[torch.cuda.Stream] = None
+                     ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Stage 3: returns (drift [H, nb, nb - budget], set_drift [H, nb]) float32."""
+    sh = _shape_of(q, block)
+    n, h = q.shape[0], q.shape[1]
+    nb = n // block
+    budget = idx.shape[-1]
+    if drift is None:
+        drift = torch.empty((h, nb, nb - budget), dtype=torch.float32, device=q.device)
+    if set_drift is None:
+        set_drift = torch.empty((h, nb), dtype=torch.float32, device=q.device)
+    need = int(lib.ress_attn_workspace_bytes(ctypes.byref(sh)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    status = lib.ress_block_drift(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(budget),
+                                  _ptr(idx), _ptr(lse), _ptr(drift) if drift.numel() else None,
+                                  _ptr(set_drift), _ptr(workspace),
+                                  0 if workspace is None else workspace.numel(),
+                                  _stream_ptr(stream, q.device))
+    _check(status, "ress_block_drift")
+    return drift, set_drift
+
+
+def ress_check_device_errors(stream: Optional[torch.cuda.Stream] = None,
+                             device: Optional[torch.device] = None) -> Tuple[int, int]:
+    """Synchronise and return (status, detail) of the device error flag (cleared)."""
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    detail = ctypes.c_int32(0)
+    status = lib.ress_check_device_errors(_stream_ptr(stream, dev), ctypes.byref(detail))
+    return int(status), int(detail.value)

@@ -1,0 +1,188 @@
+/*
+ * ress.h - C ABI of the B200 (sm_100a) block-sparse global attention library.
+ *
+ * The library implements the hot path shared by the training-free sparse
+ * global-attention methods for multi-view 3D transformers (VGGT-style):
+ *
+ *   1. ress_select_blocks      pooled block selection: mean-pool Q and K per
+ *                              block, per-head softmax over pooled logits,
+ *                              optional value-contrast term, exact-budget
+ *                              top-k per query block (ties to the lower index).
+ *   2. ress_block_sparse_attn  attention restricted to the kept key blocks.
+ *   3. ress_block_drift        per-dropped-block drift norm and drop-set drift.
+ *
+ * Sources: ReSS: Residual-Restoring Sparse Attention for 3D Vision Transformers
+ * (thelatestinai.com) - Abstract, Fig. 1, Fig. 3, Table 1, Table S5, Table S6;
+ * VASC: Value-Aware Sparse Attention with Cross-Layer Memory (paperlayer.ai) -
+ * sections 4.1, 4.2, A.1, A.2, A.3.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Tensors are token-major: q, k, v and out are [N][H][d] (d contiguous, one
+ *   token row is H*d elements).  lse is [H][N].  idx is [H][nb][budget] int32.
+ * - d must be 64.  The block size B (query blocks and key blocks alike) is 64
+ *   or 128, and N must be a multiple of B; nb = N / B.  Padding tokens, if
+ *   any, are ordinary tokens to the library.
+ * - All data pointers are device pointers owned by the caller.  The library
+ *   never allocates, frees or synchronises; every call is asynchronous and
+ *   ordered on `stream` (a cudaStream_t passed as void*, NULL = the legacy
+ *   default stream).  Scratch memory comes from the caller's `workspace`,
+ *   sized by the matching *_workspace_bytes() query, 256-byte aligned.
+ * - Argument checks run on the host before any CUDA call and return
+ *   RESS_ERR_INVALID_ARG (bad shape, NULL pointer, budget outside [1, nb],
+ *   misaligned pointer), RESS_ERR_UNSUPPORTED (valid but not implemented,
+ *   e.g. d != 64) or RESS_ERR_WORKSPACE (workspace too small).  A failed
+ *   launch returns RESS_ERR_CUDA.  When N == 0 the call returns RESS_OK and
+ *   launches nothing.
+ * - Kernels never trap.  A device-side wait that exceeds its time limit, or a
+ *   kept-block index outside [0, nb) found in a caller-provided idx (such an
+ *   index is skipped), sets a device error flag that ress_check_device_errors()
+ *   reports and clears.
+ */
+#ifndef RESS_H
+#define RESS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RESS_OK = 0,
+  RESS_ERR_INVALID_ARG = 1,
+  RESS_ERR_UNSUPPORTED = 2,
+  RESS_ERR_WORKSPACE = 3,
+  RESS_ERR_CUDA = 4,
+  RESS_ERR_TIMEOUT = 5,
+  RESS_ERR_BAD_INDEX = 6
+} ress_status;
+
+typedef enum {
+  RESS_BF16 = 0, /* bfloat16 q, k, v (and out) */
+  RESS_F32 = 1   /* float32 q, k, v (and out); attention and drift stage them to bf16 */
+} ress_dtype;
+
+typedef struct {
+  int64_t n;        /* N: tokens of all views concatenated (multiple of block) */
+  int32_t heads;    /* H: attention heads, 1..64 */
+  int32_t head_dim; /* d: must be 64 */
+  int32_t block;    /* B: 64 or 128 */
+  int32_t dtype;    /* ress_dtype of q, k and v */
+} ress_shape;
+
+/* Library version, (major << 16) | minor. */
+int ress_version(void);
+
+/* Human-readable name of a status code; never NULL. */
+const char* ress_status_string(ress_status status);
+
+/*
+ * Workspace bytes that ress_select_blocks needs for `shape` and `lambda`
+ * (0 if the shape is invalid).  Layout, all float32, each array 256-byte
+ * aligned, in this order: Qbar [H][nb][64], Kbar^T [H][64][nb_pad],
+ * Vbar [H][nb][64] (lambda > 0 only), contrast [H][nb] (lambda > 0 only),
+ * with nb_pad = nb rounded up to 256.
+ */
+size_t ress_select_workspace_bytes(const ress_shape* shape, float lambda);
+
+/*
+ * Stage 1: pooled block selection (ReSS Table S5, SpargeAttn row: pooled
+ * query/key inner products; VASC 4.1: pooled relevance plus neighbouring
+ * value contrast; VASC A.2: an exact-capacity binary Top-K mask).
+ *
+ * For each head h and query block i:
+ *   Qbar_i = mean of the B query tokens of block i (same for Kbar_j, Vbar_j),
+ *   s_ij   = (Qbar_i . Kbar_j) / sqrt(d),
+ *   p_ij   = softmax over all nb key blocks j of s_ij,
+ *   c_j    = ||Vbar_j - Vbar_{j-1}||_2 for j >= 1, c_0 = 0,
+ *   score  = p_ij + lambda * c_j,
+ * and idx[h][i][0..budget) receives the `budget` blocks of largest score in
+ * ascending block order; equal scores go to the lower block index.  With
+ * lambda == 0 the ranking uses s_ij, which orders the row as p_ij does.
+ *
+ *   q, k    [N][H][64] of shape->dtype, 16-byte aligned.
+ *   v       [N][H][64], read only when lambda > 0 (may be NULL otherwise).
+ *   budget  kept key blocks per query block, 1 <= budget <= nb.
+ *   lambda  contrast weight, finite and >= 0.
+ *   idx     out, [H][nb][budget] int32.
+ *   Supported sizes: nb <= 4096.
+ */
+ress_status ress_select_blocks(const ress_shape* shape, const void* q, const void* k,
+                               const void* v, int32_t budget, float lambda, int32_t* idx,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Workspace bytes that ress_block_sparse_attn and ress_block_drift need:
+ * 0 for bf16 inputs; 3 * N * H * 64 * 2 for float32 inputs (bf16 copies of
+ * q, k and v).
+ */
+size_t ress_attn_workspace_bytes(const ress_shape* shape);
+
+/*
+ * Stage 2: block-sparse attention forward (ReSS Table S6: the selection feeds
+ * one shared block-sparse kernel on the block grid; VASC 4.2: the binary mask
+ * is passed directly to the sparse kernel; ReSS Table S5: bidirectional, no
+ * causal mask).
+ *
+ * For query token n of block i and head h, with kept set K(h, i) = idx[h][i]:
+ *   out[n][h] = sum_{t in K} softmax_t((q[n][h] . k[t][h]) / sqrt(d)) v[t][h],
+ * normalised over the kept tokens only, and
+ *   lse[h][n] = ln sum_{t in K} exp((q[n][h] . k[t][h]) / sqrt(d)).
+ *
+ *   idx    [H][nb][budget] int32 device array; rows need not be sorted or
+ *          unique (duplicates count once); entries outside [0, nb) are skipped
+ *          and flagged (RESS_ERR_BAD_INDEX via ress_check_device_errors).
+ *   out        [N][H][64] of `out_dtype` (RESS_BF16 or RESS_F32, independent
+ *              of the input dtype).
+ *   lse        [H][N] float32, or NULL.
+ *   The contractions run on bf16 operands with float32 accumulation; the
+ *   probabilities enter P V as bf16 and the row normaliser is the sum of those
+ *   same bf16 values, so each output row is a convex combination of kept
+ *   values.  lse uses the float32 probabilities.
+ */
+ress_status ress_block_sparse_attn(const ress_shape* shape, const void* q, const void* k,
+                                   const void* v, int32_t budget, const int32_t* idx,
+                                   void* out, int32_t out_dtype, float* lse, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/*
+ * Stage 3: drift of the dropped blocks (ReSS Abstract and Fig. 3: the drift
+ * score measures how much masking a block shifts what attention writes into
+ * the residual stream; the drift of a drop set depends on the directions of
+ * the contributions, Fig. 9 plots quality against it).
+ *
+ * For query block i of head h and every dropped block j (not in idx[h][i]),
+ * in ascending j order r = 0 .. nb - budget - 1:
+ *   C_j[n][:] = sum_{t in block j} exp((q[n] . k[t]) / sqrt(d) - lse[h][n]) v[t][:]
+ *   drift[h][i][r] = ||C_j||_F over the B x 64 matrix,
+ *   set_drift[h][i] = || sum_{j dropped} C_j ||_F.
+ * lse is the kept-set normaliser written by ress_block_sparse_attn for the
+ * same idx.
+ *
+ *   idx        as for ress_block_sparse_attn, but rows must hold `budget`
+ *              distinct in-range blocks (the drift row length is nb - budget).
+ *   lse        [H][N] float32 from ress_block_sparse_attn.
+ *   drift      out, [H][nb][nb - budget] float32 (may be NULL when budget == nb).
+ *   set_drift  out, [H][nb] float32, or NULL.
+ */
+ress_status ress_block_drift(const ress_shape* shape, const void* q, const void* k,
+                             const void* v, int32_t budget, const int32_t* idx,
+                             const float* lse, float* drift, float* set_drift,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reports and clears the device error flag that
+ * the kernels set: RESS_ERR_TIMEOUT (a device wait ran out of time),
+ * RESS_ERR_BAD_INDEX (an idx entry outside [0, nb) was skipped), RESS_OK if
+ * none, RESS_ERR_CUDA if the synchronisation itself failed.  `detail`, if not
+ * NULL, receives a kernel-specific code of the first error (0 if none).
+ */
+ress_status ress_check_device_errors(void* stream, int32_t* detail);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RESS_H */

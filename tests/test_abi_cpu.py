@@ -1,0 +1,137 @@
+"""The C-ABI library loads, exports every entry point that include/ress.h
+declares, and rejects bad arguments on the host before any CUDA call (these
+cases need no GPU)."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from block_sparse_global_mean_b200 import build as ress_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ress.h")
+
+
+@pytest.fixture(scope="module")
+def ress():
+    ress_build.build()
+    from block_sparse_global_mean_b200 import ress as mod
+    return mod
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ress_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_three_stage_entry_points():
+    names = _declared_functions()
+    for n in ("ress_select_blocks", "ress_block_sparse_attn", "ress_block_drift"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(ress):
+    names = _declared_functions()
+    out = subprocess.run(["nm", "-D", "--defined-only", ress.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\bT\s+(\w+)$", out, flags=re.M))
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    for n in names:
+        assert hasattr(ress.lib, n)
+
+
+def test_library_is_built_for_sm100a(ress):
+    out = subprocess.run(["strings", ress.LIB_PATH], capture_output=True, text=True).stdout
+    assert "sm_100a" in out
+
+
+def test_status_strings(ress):
+    assert ress.lib.ress_status_string(0) == b"ok"
+    assert ress.lib.ress_status_string(3) == b"workspace too small"
+    assert ress.lib.ress_status_string(99) == b"unknown status"
+    assert ress.lib.ress_version() >> 16 == 1
+
+
+def _shape(ress, n=512, heads=2, d=64, block=64, dtype=0):
+    return ress.ress_shape(n, heads, d, block, dtype)
+
+
+FAKE = 0x10000          # 16-byte aligned, never dereferenced: every case fails validation
+FAKE_WS = 0x20000       # 256-byte aligned
+
+
+def _select(ress, shape, q=FAKE, k=FAKE, v=None, budget=4, lam=0.0, idx=FAKE, ws=FAKE_WS,
+            ws_bytes=1 << 30):
+    return ress.lib.ress_select_blocks(ctypes.byref(shape) if shape is not None else None, q, k, v,
+                                       budget, ctypes.c_float(lam), idx, ws, ws_bytes, None)
+
+
+def test_select_rejects_bad_arguments_on_the_host(ress):
+    E = ress
+    assert _select(ress, None) == E.RESS_ERR_INVALID_ARG
+    assert _select(ress, _shape(ress, d=32)) == E.RESS_ERR_UNSUPPORTED
+    assert _select(ress, _shape(ress, block=96)) == E.RESS_ERR_UNSUPPORTED
+    assert _select(ress, _shape(ress, n=500)) == E.RESS_ERR_INVALID_ARG      # not a multiple of B
+    assert _select(ress, _shape(ress, heads=0)) == E.RESS_ERR_INVALID_ARG
+    assert _select(ress, _shape(ress, heads=65)) == E.RESS_ERR_UNSUPPORTED
+    assert _select(ress, _shape(ress, dtype=7)) == E.RESS_ERR_INVALID_ARG
+    assert _select(ress, _shape(ress), budget=0) == E.RESS_ERR_INVALID_ARG
+    assert _select(ress, _shape(ress), budget=9) == E.RESS_ERR_INVALID_ARG   # nb = 8
+    assert _select(ress, _shape(ress), lam=-1.0) == E.RESS_ERR_INVALID_ARG
+    assert _select(ress, _shape(ress), lam=float("nan")) == E.RESS_ERR_INVALID_ARG
+    assert _select(ress, _shape(ress), lam=0.5, v=None) == E.RESS_ERR_INVALID_ARG
+    assert _select(ress, _shape(ress), q=None) == E.RESS_ERR_INVALID_ARG
+    assert _select(ress, _shape(ress), q=FAKE + 8) == E.RESS_ERR_INVALID_ARG  # misaligned
+    assert _select(ress, _shape(ress), ws=FAKE_WS + 16) == E.RESS_ERR_INVALID_ARG
+    assert _select(ress, _shape(ress), ws_bytes=16) == E.RESS_ERR_WORKSPACE
+    big = _shape(ress, n=64 * 4097)
+    assert _select(ress, big, budget=1) == E.RESS_ERR_UNSUPPORTED               # nb > 4096
+
+
+def test_empty_input_is_a_no_op(ress):
+    sh = _shape(ress, n=0)
+    assert _select(ress, sh, budget=0) == ress.RESS_OK
+    assert ress.lib.ress_block_sparse_attn(ctypes.byref(sh), FAKE, FAKE, FAKE, 0, FAKE, FAKE, 0,
+                                           None, None, 0, None) == ress.RESS_OK
+    assert ress.lib.ress_block_drift(ctypes.byref(sh), FAKE, FAKE, FAKE, 0, FAKE, FAKE, FAKE,
+                                     None, None, 0, None) == ress.RESS_OK
+
+
+def test_attention_and_drift_reject_bad_arguments_on_the_host(ress):
+    sh = _shape(ress)
+    lib = ress.lib
+    assert lib.ress_block_sparse_attn(ctypes.byref(sh), FAKE, FAKE, FAKE, 0, FAKE, FAKE, 0,
+                                      None, None, 0, None) == ress.RESS_ERR_INVALID_ARG
+    assert lib.ress_block_sparse_attn(ctypes.byref(sh), FAKE, FAKE, None, 4, FAKE, FAKE, 0,
+                                      None, None, 0, None) == ress.RESS_ERR_INVALID_ARG
+    assert lib.ress_block_sparse_attn(ctypes.byref(sh), FAKE, FAKE, FAKE, 4, FAKE + 2, FAKE, 0,
+                                      None, None, 0, None) == ress.RESS_ERR_INVALID_ARG
+    assert lib.ress_block_sparse_attn(ctypes.byref(sh), FAKE, FAKE, FAKE, 4, FAKE, FAKE, 5,
+                                      None, None, 0, None) == ress.RESS_ERR_INVALID_ARG  # out dtype
+    f32 = _shape(ress, dtype=1)
+    assert lib.ress_block_sparse_attn(ctypes.byref(f32), FAKE, FAKE, FAKE, 4, FAKE, FAKE, 0,
+                                      None, None, 0, None) == ress.RESS_ERR_WORKSPACE
+    assert lib.ress_block_drift(ctypes.byref(sh), FAKE, FAKE, FAKE, 4, FAKE, None, FAKE, None,
+                                None, 0, None) == ress.RESS_ERR_INVALID_ARG     # lse NULL
+    assert lib.ress_block_drift(ctypes.byref(sh), FAKE, FAKE, FAKE, 4, FAKE, FAKE, None, None,
+                                None, 0, None) == ress.RESS_ERR_INVALID_ARG     # drift NULL
+    assert lib.ress_block_drift(ctypes.byref(sh), FAKE, FAKE, FAKE, 9, FAKE, FAKE, FAKE, None,
+                                None, 0, None) == ress.RESS_ERR_INVALID_ARG     # budget > nb
+
+
+def test_workspace_queries(ress):
+    import torch
+    # bf16, 100 views x 1,408 tokens, H=16, B=64, lambda=0: Qbar + Kbar^T (nb_pad 2304)
+    n, h, nb = 140800, 16, 2200
+    got = ress.select_workspace_bytes(n, h, 64, torch.bfloat16, 0.0)
+    assert got == 4 * h * nb * 64 + 4 * h * 64 * 2304
+    with_v = ress.select_workspace_bytes(n, h, 64, torch.bfloat16, 0.5)
+    assert with_v == got + 4 * h * nb * 64 + 4 * h * nb
+    assert ress.attn_workspace_bytes(n, h, 64, torch.bfloat16) == 0
+    assert ress.attn_workspace_bytes(512, 2, 64, torch.float32) == 3 * 512 * 2 * 64 * 2
+    assert ress.lib.ress_select_workspace_bytes(None, ctypes.c_float(0.0)) == 0
