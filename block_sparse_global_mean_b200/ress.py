@@ -61,6 +61,8 @@ lib.ress_block_sparse_attn.argtypes = [_SHAPE, _P, _P, _P, ctypes.c_int32, _P, _
 lib.ress_block_drift.restype = ctypes.c_int
 lib.ress_block_drift.argtypes = [_SHAPE, _P, _P, _P, ctypes.c_int32, _P, _P, _P, _P, _P,
                                  ctypes.c_size_t, _P]
+lib.ress_select_blocks_noalloc.restype = ctypes.c_int
+lib.ress_select_blocks_noalloc.argtypes = [_SHAPE, _P, _P, _P, ctypes.c_int32, ctypes.c_float, _P, _P]
 lib.ress_check_device_errors.restype = ctypes.c_int
 lib.ress_check_device_errors.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
 
@@ -136,6 +138,23 @@ def ress_select_blocks(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tenso
                                     ctypes.c_float(lam), _ptr(idx), _ptr(workspace),
                                     workspace.numel(), _stream_ptr(stream, q.device))
     _check(status, "ress_select_blocks")
+    return idx
+
+
+def ress_select_blocks_noalloc(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor],
+                               budget: int, lam: float, block: int,
+                               idx: Optional[torch.Tensor] = None,
+                               stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Stage 1 with the library's fixed scratch array instead of a workspace
+    (for callers that cannot allocate device memory); see include/ress.h."""
+    sh = _shape_of(q, block)
+    n, h = q.shape[0], q.shape[1]
+    if idx is None:
+        idx = torch.empty((h, n // block, budget), dtype=torch.int32, device=q.device)
+    status = lib.ress_select_blocks_noalloc(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(budget),
+                                            ctypes.c_float(lam), _ptr(idx),
+                                            _stream_ptr(stream, q.device))
+    _check(status, "ress_select_blocks_noalloc")
     return idx
 
 

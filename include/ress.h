@@ -114,6 +114,32 @@ ress_status ress_select_blocks(const ress_shape* shape, const void* q, const voi
                                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Stage 1 for callers that cannot allocate device memory.  The pages have no
+ * counterpart to this entry point; it exists for callers that may not call
+ * cudaMalloc or hold a workspace of their own (for example a plugin running
+ * inside another framework's allocator, or a loop in which an allocation,
+ * which can synchronise the device, is not allowed).
+ *
+ * Same arguments, checks and result as ress_select_blocks, without the
+ * workspace: the scratch lives in one fixed 32 MiB array in device memory
+ * that the library owns (H = 16 and nb <= 2,200 fit, with the value
+ * contrast).  Every GPU that loads the library holds that array until the
+ * process exits.  A problem whose ress_select_workspace_bytes() exceeds
+ * 32 MiB is rejected with RESS_ERR_WORKSPACE before anything is launched.
+ *
+ * - The first call on a device looks up the array's device address (one
+ *   cudaGetSymbolAddress with that device current); make that first call
+ *   before any stream capture.  The call allocates nothing.
+ * - All calls share the one array, and each call overwrites every scratch
+ *   value it reads, so nothing needs to start at zero.  Calls that overlap on
+ *   the GPU (different streams, or different host threads, on one device)
+ *   race on the array and must be ordered by the caller.
+ */
+ress_status ress_select_blocks_noalloc(const ress_shape* shape, const void* q, const void* k,
+                                       const void* v, int32_t budget, float lambda,
+                                       int32_t* idx, void* stream);
+
+/*
  * Workspace bytes that ress_block_sparse_attn and ress_block_drift need:
  * 0 for bf16 inputs; 3 * N * H * 64 * 2 for float32 inputs (bf16 copies of
  * q, k and v).
