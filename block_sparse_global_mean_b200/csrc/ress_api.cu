@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <cmath>
+#include <cstdio>
 #include <mutex>
 
 #include "ress_common.cuh"
@@ -69,6 +70,17 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 
 }  // namespace
 
+namespace {
+thread_local char g_last_cuda_error[256] = "";
+}  // namespace
+
+ress_status record_cuda(cudaError_t err) {
+  if (err == cudaSuccess) return RESS_OK;
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", cudaGetErrorName(err),
+           cudaGetErrorString(err));
+  return RESS_ERR_CUDA;
+}
+
 DeviceError* device_error_ptr() {
   // One address per device; looked up with that device current.
   static DeviceError* cache[64] = {};
@@ -78,7 +90,7 @@ DeviceError* device_error_ptr() {
   std::lock_guard<std::mutex> lock(mu);
   if (cache[dev] == nullptr) {
     void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_device_error) != cudaSuccess) return nullptr;
+    if (record_cuda(cudaGetSymbolAddress(&ptr, g_device_error)) != RESS_OK) return nullptr;
     cache[dev] = static_cast<DeviceError*>(ptr);
   }
   return cache[dev];
@@ -95,6 +107,9 @@ bool make_token_map(CUtensorMap* map, const void* base, const Geometry& g, int r
                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+             "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
   return r == CUDA_SUCCESS;
 }
 
@@ -104,7 +119,7 @@ ress_status launch_cast_bf16(const float* src, __nv_bfloat16* dst, size_t count,
   const unsigned blocks = (unsigned)((n4 + 255) / 256 < 148 * 16 ? (n4 + 255) / 256 : 148 * 16);
   cast_bf16_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(src),
                                            reinterpret_cast<uint2*>(dst), n4);
-  return cudaGetLastError() == cudaSuccess ? RESS_OK : RESS_ERR_CUDA;
+  return record_cuda(cudaGetLastError());
 }
 
 }  // namespace ress
@@ -229,17 +244,19 @@ ress_status ress_block_drift(const ress_shape* shape, const void* q, const void*
 
 ress_status ress_check_device_errors(void* stream, int32_t* detail) {
   if (detail) *detail = 0;
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return RESS_ERR_CUDA;
+  if (ress_status s = record_cuda(cudaStreamSynchronize(static_cast<cudaStream_t>(stream))))
+    return s;
   DeviceError e{0, 0};
-  if (cudaMemcpyFromSymbol(&e, g_device_error, sizeof(e)) != cudaSuccess) return RESS_ERR_CUDA;
+  if (ress_status s = record_cuda(cudaMemcpyFromSymbol(&e, g_device_error, sizeof(e)))) return s;
   if (e.code != 0) {
     const DeviceError zero{0, 0};
-    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess)
-      return RESS_ERR_CUDA;
+    if (ress_status s = record_cuda(cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero))))
+      return s;
   }
   if (detail) *detail = e.detail;
   return static_cast<ress_status>(e.code);
 }
+
+const char* ress_last_cuda_error(void) { return g_last_cuda_error; }
 
 }  // extern "C"

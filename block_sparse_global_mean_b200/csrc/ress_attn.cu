@@ -8,15 +8,24 @@
 // tokens only (ReSS Table S6 / VASC 4.2: the selection's binary block mask
 // drives one shared sparse kernel; ReSS Table S5: no causal mask).
 //
-// Warp roles (192 threads, two CTAs per SM):
+// Warp roles (320 threads, one CTA per SM):
 //   warp 0     TMA producer: Q tile once, then K/V sub-blocks of each chunk
-//              into a 2-stage ring (128-byte swizzle).
+//              into a 4-stage ring (128-byte swizzle).
 //   warp 1     TMEM owner and MMA issuer: S = Q K^T (M=128, N=128, K=64) into
-//              TMEM, then O += P V (M=128, N=64, K=128) with P read from TMEM.
-//   warps 2-5  softmax: one query row per thread; S from TMEM, online softmax
-//              in the log2 domain with a lazy rescale of O (only when the
-//              running maximum grows by more than 2^8), P written back to TMEM
-//              as bf16 over the first 64 columns of S; epilogue O / sum(P) and lse.
+//              one of two TMEM buffers, so S of chunk c+1 is computed while the
+//              softmax warps work on chunk c; then O += P V (M=128, N=64,
+//              K=128) with P read from TMEM.
+//   warps 2-9  softmax, one query row per thread, in two groups: warps 2-5
+//              take the even chunks and warps 6-9 the odd ones, each group with
+//              its own running maximum, sums and O accumulator in TMEM (a
+//              split over chunks, merged in the epilogue), so one group's
+//              TMEM and barrier latency overlaps the other's exponentials.
+//              S is read from TMEM, the online softmax runs in the log2 domain
+//              with a lazy rescale of O (only when the running maximum grows
+//              by more than 2^8), and P goes back to TMEM as bf16 over the
+//              first 64 columns of S; epilogue O / sum(P) and lse.
+//              The row sums of the bf16 P come from one more MMA, P times a
+//              16-column tile of ones (N=16), accumulated next to O.
 //
 // Every mbarrier wait is bounded; on timeout the CTA raises the device error,
 // drains its copies and MMAs in flight, frees TMEM and exits.
@@ -28,14 +37,18 @@ namespace ress {
 namespace {
 
 constexpr int kRows = 128;
-constexpr int kStages = 2;
-constexpr int kThreads = 192;
+constexpr int kStages = 4;
+constexpr int kThreads = 320;
 constexpr uint32_t kQBytes = 128 * 128;            // 128 rows x 64 bf16
 constexpr uint32_t kSubBytes = 64 * 128;           // 64 keys x 64 bf16
 constexpr uint32_t kStageBytes = 4 * kSubBytes;    // K sub0, K sub1, V sub0, V sub1
-constexpr uint32_t kTmemCols = 256;
-constexpr uint32_t kColS = 0;                      // S: 128 fp32 columns; P: bf16 in cols 0..63
-constexpr uint32_t kColO = 128;                    // O: 64 fp32 columns
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0;                      // S buffers at 0 and 128 (128 fp32 columns each;
+                                                   // P as bf16 in the first 64 columns of its buffer)
+constexpr uint32_t kColO = 256;                    // O of the even / odd chunks: 2 x 64 fp32 columns
+constexpr uint32_t kColL = 384;                    // row sums of the bf16 P (P times a ones tile),
+                                                   // even / odd chunks: 2 x 16 columns
+constexpr uint32_t kOnesBytes = 16 * 128;          // 16 x 64 bf16 ones, K-major, 128-byte swizzle
 
 struct AttnParams {
   DeviceError* err;
@@ -54,20 +67,23 @@ struct __align__(8) Ctl {
   uint64_t q_full;
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
-  uint64_t s_full;
-  uint64_t p_full;
+  uint64_t s_full[2];   // S buffer b holds S of chunk c (c % 2 == b)
+  uint64_t p_full[2];   // P of chunk c written into S buffer c % 2
   uint64_t o_full;
+  uint64_t merge;       // the odd-chunk group posted its row statistics
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
   int n_entries;
   int pad;
+  float odd_m[kRows];   // odd-chunk group: reference maximum (log2 domain) per row
+  float odd_l[kRows];   // odd-chunk group: float32 probability sum per row
 };
 
 __host__ __device__ inline int words_for(int nb) { return (nb + 31) >> 5; }
 
 size_t attn_smem_bytes(int nb) {
-  return 1024 + kQBytes + kStages * kStageBytes + sizeof(Ctl) +
+  return 1024 + kQBytes + kStages * kStageBytes + kOnesBytes + sizeof(Ctl) +
          sizeof(uint32_t) * (2 * (size_t)words_for(nb) + (size_t)nb);
 }
 
@@ -103,6 +119,33 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 template <typename OutT>
+__device__ __forceinline__ void store_half_row(OutT* dst, const float* o, float inv);
+
+template <>
+__device__ __forceinline__ void store_half_row<__nv_bfloat16>(__nv_bfloat16* dst, const float* o,
+                                                              float inv) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    uint4 v;
+    v.x = pack_bf16x2(o[8 * u + 0] * inv, o[8 * u + 1] * inv);
+    v.y = pack_bf16x2(o[8 * u + 2] * inv, o[8 * u + 3] * inv);
+    v.z = pack_bf16x2(o[8 * u + 4] * inv, o[8 * u + 5] * inv);
+    v.w = pack_bf16x2(o[8 * u + 6] * inv, o[8 * u + 7] * inv);
+    d4[u] = v;
+  }
+}
+
+template <>
+__device__ __forceinline__ void store_half_row<float>(float* dst, const float* o, float inv) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int u = 0; u < 8; ++u)
+    d4[u] = make_float4(o[4 * u] * inv, o[4 * u + 1] * inv, o[4 * u + 2] * inv,
+                        o[4 * u + 3] * inv);
+}
+
+template <typename OutT>
 __device__ __forceinline__ void store_row(OutT* dst, const float* o, float inv);
 
 template <>
@@ -129,8 +172,10 @@ __device__ __forceinline__ void store_row<float>(float* dst, const float* o, flo
                         o[4 * u + 3] * inv);
 }
 
+// 10 warps: three of them share an SM sub-partition's 16,384 registers, so
+// the launch bound caps the kernel at 168 registers per thread.
 template <typename OutT>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                              const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -139,7 +184,8 @@ __global__ void __launch_bounds__(kThreads, 2)
                                              ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + kQBytes;
-  Ctl* ctl = reinterpret_cast<Ctl*>(sKV + kStages * kStageBytes);
+  uint8_t* sOnes = sKV + kStages * kStageBytes;
+  Ctl* ctl = reinterpret_cast<Ctl*>(sOnes + kOnesBytes);
   const int W = words_for(p.nb);
   uint32_t* bmA = reinterpret_cast<uint32_t*>(ctl + 1);
   uint32_t* bmB = bmA + W;
@@ -154,9 +200,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int qb0 = (p.block == 64) ? 2 * tile : tile;
 
   const uint32_t bar_q = smem_addr(&ctl->q_full);
-  const uint32_t bar_s = smem_addr(&ctl->s_full);
-  const uint32_t bar_p = smem_addr(&ctl->p_full);
+  const uint32_t bar_s0 = smem_addr(&ctl->s_full[0]);
+  const uint32_t bar_p0 = smem_addr(&ctl->p_full[0]);
   const uint32_t bar_o = smem_addr(&ctl->o_full);
+  const uint32_t bar_merge = smem_addr(&ctl->merge);
   const uint32_t bar_done = smem_addr(&ctl->mma_done);
   volatile int* abortf = &ctl->abort_flag;
 
@@ -166,9 +213,12 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(smem_addr(&ctl->kv_full[s]), 1);
       mbar_init(smem_addr(&ctl->kv_empty[s]), 1);
     }
-    mbar_init(bar_s, 1);
-    mbar_init(bar_p, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_s0 + 8 * b, 1);
+      mbar_init(bar_p0 + 8 * b, 128);
+    }
     mbar_init(bar_o, 1);
+    mbar_init(bar_merge, 128);
     mbar_init(bar_done, 1);
     ctl->abort_flag = 0;
     fence_mbarrier_init();
@@ -178,6 +228,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     tmem_relinquish();
   }
   for (int w = threadIdx.x; w < 2 * W; w += kThreads) bmA[w] = 0u;
+  // bf16 ones: the B operand of the MMA that sums each row of P.
+  for (int w = threadIdx.x; w < (int)(kOnesBytes / 4); w += kThreads)
+    reinterpret_cast<uint32_t*>(sOnes)[w] = 0x3F803F80u;
+  fence_proxy_async_smem();
   __syncthreads();
 
   // Kept sets of the tile's query blocks as bitmaps (duplicates collapse,
@@ -231,29 +285,35 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int n_chunks = (p.block == 64) ? (n_entries + 1) / 2 : n_entries;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0 && n_chunks > 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar_q, kQBytes);
-      tma_load_3d(smem_addr(sQ), &tm_q, bar_q, 0, h, row0);
+    // ---------------- TMA producer (whole warp; one elected lane issues) ----------------
+    if (n_chunks > 0) {
+      if (elect_one()) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        mbar_arrive_expect_tx(bar_q, kQBytes);
+        tma_load_3d(smem_addr(sQ), &tm_q, bar_q, 0, h, row0);
+      }
+      __syncwarp();
       int issued = 0;
       for (int c = 0; c < n_chunks; ++c) {
         const int s = c % kStages;
         if (c >= kStages &&
-            !mbar_wait(smem_addr(&ctl->kv_empty[s]), ((c / kStages) - 1) & 1, abortf, p.err, 10))
+            !warp_wait(smem_addr(&ctl->kv_empty[s]), ((c / kStages) - 1) & 1, abortf, p.err, 10))
           break;
         int t0, t1;
         uint32_t m0, m1;
         chunk_info(list, n_entries, p.block, c, t0, t1, m0, m1);
-        uint8_t* st = sKV + s * kStageBytes;
+        const uint32_t st = smem_addr(sKV) + (uint32_t)s * kStageBytes;
         const uint32_t bar = smem_addr(&ctl->kv_full[s]);
-        mbar_arrive_expect_tx(bar, kStageBytes);
-        tma_load_3d(smem_addr(st), &tm_k, bar, 0, h, t0);
-        tma_load_3d(smem_addr(st + kSubBytes), &tm_k, bar, 0, h, t1);
-        tma_load_3d(smem_addr(st + 2 * kSubBytes), &tm_v, bar, 0, h, t0);
-        tma_load_3d(smem_addr(st + 3 * kSubBytes), &tm_v, bar, 0, h, t1);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar, kStageBytes);
+          tma_load_3d(st, &tm_k, bar, 0, h, t0);
+          tma_load_3d(st + kSubBytes, &tm_k, bar, 0, h, t1);
+          tma_load_3d(st + 2 * kSubBytes, &tm_v, bar, 0, h, t0);
+          tma_load_3d(st + 3 * kSubBytes, &tm_v, bar, 0, h, t1);
+        }
+        __syncwarp();
         issued = c + 1;
       }
       // Copies still in flight must land before the CTA can exit.
@@ -263,68 +323,100 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0 && n_chunks > 0) {
+    // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
+    if (n_chunks > 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idPV = idesc_bf16_f32(128, 64, true);
+      constexpr uint32_t idL = idesc_bf16_f32(128, 16, false);
       const uint32_t tS = tmem + kColS;
       const uint32_t tO = tmem + kColO;
+      const uint32_t tL = tmem + kColL;
+      const uint64_t dones = smem_desc_sw128(smem_addr(sOnes), 16, 1024);
       const uint64_t dq = smem_desc_sw128(smem_addr(sQ), 16, 1024);
-      bool ok = mbar_wait(bar_q, 0, abortf, p.err, 20);
+      // Stage s: K at +s*kStageBytes, V at +2*kSubBytes; one 16-key step of V
+      // is 2048 bytes (128 units of 16 bytes in the descriptor's address field).
+      const uint64_t dk0 = smem_desc_sw128(smem_addr(sKV), 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(smem_addr(sKV) + 2 * kSubBytes, 16384, 1024);
+      constexpr uint64_t kStageDesc = kStageBytes >> 4;
+      bool ok = warp_wait(bar_q, 0, abortf, p.err, 20);
+      auto issue_s = [&](int c) -> bool {
+        const int s = c % kStages;
+        if (!warp_wait(smem_addr(&ctl->kv_full[s]), (c / kStages) & 1, abortf, p.err, 22))
+          return false;
+        tc_fence_after();
+        const uint64_t dk = dk0 + (uint64_t)s * kStageDesc;
+        const uint32_t tSb = tS + 128u * (uint32_t)(c & 1);
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tSb, dq + (uint64_t)(kk * 2), dk + (uint64_t)(kk * 2), idS, kk > 0 ? 1u : 0u);
+          mma_commit(bar_s0 + 8u * (uint32_t)(c & 1));
+        }
+        __syncwarp();
+        return true;
+      };
       auto issue_pv = [&](int c) {
         const int sp = c % kStages;
-        const uint32_t vaddr = smem_addr(sKV + sp * kStageBytes + 2 * kSubBytes);
+        const uint64_t dv = dv0 + (uint64_t)sp * kStageDesc;
+        const uint32_t par = (uint32_t)(c & 1);
+        const uint32_t tP = tS + 128u * par;
+        const uint32_t tOp = tO + 64u * par;
+        const uint32_t tLp = tL + 16u * par;
+        const uint32_t acc0 = c > 1 ? 1u : 0u;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t dv = smem_desc_sw128(vaddr + kk * 2048, 16384, 1024);
-          mma_ts(tO, tS + kk * 8, dv, idPV, (c > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tOp, tP + kk * 8, dv + (uint64_t)(kk * 128), idPV, kk > 0 ? 1u : acc0);
+          // Row sums of the same bf16 P: every 16-key slice of the ones tile is 1.
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) mma_ts(tLp, tP + kk * 8, dones, idL, kk > 0 ? 1u : acc0);
+          mma_commit(smem_addr(&ctl->kv_empty[sp]));
         }
-        mma_commit(smem_addr(&ctl->kv_empty[sp]));
+        __syncwarp();
       };
+      if (ok) ok = issue_s(0);
       for (int c = 0; ok && c < n_chunks; ++c) {
-        if (c > 0) {
-          // P(c-1) must be consumed before S(c) overwrites its columns; the
-          // tensor core runs this thread's MMAs in issue order.
-          if (!mbar_wait(bar_p, (c - 1) & 1, abortf, p.err, 21)) { ok = false; break; }
-          tc_fence_after();
-          issue_pv(c - 1);
-        }
-        const int s = c % kStages;
-        if (!mbar_wait(smem_addr(&ctl->kv_full[s]), (c / kStages) & 1, abortf, p.err, 22)) {
+        // S(c+1) goes to the other buffer, which holds P(c-1): PV(c-1) was
+        // issued before it, and the tensor core runs the MMAs in issue order.
+        if (c + 1 < n_chunks && !(ok = issue_s(c + 1))) break;
+        if (!warp_wait(bar_p0 + 8u * (uint32_t)(c & 1), (c >> 1) & 1, abortf, p.err, 21)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint64_t dk = smem_desc_sw128(smem_addr(sKV + s * kStageBytes), 16, 1024);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tS, dq + (uint64_t)(kk * 2), dk + (uint64_t)(kk * 2), idS, kk > 0 ? 1u : 0u);
-        mma_commit(bar_s);
+        issue_pv(c);
       }
-      if (ok && mbar_wait(bar_p, (n_chunks - 1) & 1, abortf, p.err, 23)) {
-        tc_fence_after();
-        issue_pv(n_chunks - 1);
-        mma_commit(bar_o);
+      if (elect_one()) {
+        if (ok) mma_commit(bar_o);
+        mma_commit(bar_done);
       }
-      mma_commit(bar_done);
+      __syncwarp();
       mbar_wait_drain(bar_done, 0, p.err, 24);
     }
     __syncwarp();
   } else {
-    // ---------------- softmax + epilogue (warps 2..5) ----------------
+    // ---------------- softmax + epilogue (warps 2..9) ----------------
     const int quad = warp & 3;             // TMEM lanes 32*quad .. 32*quad+31
+    const int par = (warp - 2) >> 2;       // 0: even chunks, 1: odd chunks
     const int row = quad * 32 + lane;
     const int half = row >> 6;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t tS = tmem + kColS + lane_off;
-    const uint32_t tO = tmem + kColO + lane_off;
+    const uint32_t tS = tmem + kColS + lane_off + 128u * (uint32_t)par;
+    const uint32_t tO = tmem + kColO + lane_off + 64u * (uint32_t)par;
+    const uint32_t tL = tmem + kColL + lane_off + 16u * (uint32_t)par;
+    const uint32_t bar_s = bar_s0 + 8u * (uint32_t)par;
+    const uint32_t bar_p = bar_p0 + 8u * (uint32_t)par;
     const float kScaleLog2 = 1.4426950408889634f * 0.125f;   // log2(e) / sqrt(64)
+    const float2 scale2 = make_float2(kScaleLog2, kScaleLog2);
     float m_ref = -INFINITY;
-    float l = 0.f;    // sum of the float32 probabilities (for lse)
-    float lr = 0.f;   // sum of the same probabilities rounded to bf16 (normaliser of P V)
+    float2 l2 = make_float2(0.f, 0.f);   // float32 probability sums (for lse)
+    float2 l2b = make_float2(0.f, 0.f);
     bool ok = true;
-    for (int c = 0; c < n_chunks; ++c) {
-      if (!warp_wait(bar_s, c & 1, abortf, p.err, 30)) { ok = false; break; }
+    for (int c = par, it = 0; c < n_chunks; c += 2, ++it) {
+      if (!warp_wait(bar_s, it & 1, abortf, p.err, 30)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       int t0, t1;
       uint32_t m0, m1;
@@ -348,42 +440,38 @@ __global__ void __launch_bounds__(kThreads, 2)
       tmem_ld32(tS + 64, r[2]);
       tmem_ld32(tS + 96, r[3]);
       tmem_ld_wait();
-      float mx = -INFINITY;
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
       if (use0) {
 #pragma unroll
-        for (int u = 0; u < 32; ++u) mx = fmaxf(mx, fmaxf(__uint_as_float(r[0][u]), __uint_as_float(r[1][u])));
+        for (int u = 0; u < 16; ++u) {
+          mx0 = fmax3(mx0, __uint_as_float(r[0][2 * u]), __uint_as_float(r[0][2 * u + 1]));
+          mx1 = fmax3(mx1, __uint_as_float(r[1][2 * u]), __uint_as_float(r[1][2 * u + 1]));
+        }
       }
       if (use1) {
 #pragma unroll
-        for (int u = 0; u < 32; ++u) mx = fmaxf(mx, fmaxf(__uint_as_float(r[2][u]), __uint_as_float(r[3][u])));
+        for (int u = 0; u < 16; ++u) {
+          mx2 = fmax3(mx2, __uint_as_float(r[2][2 * u]), __uint_as_float(r[2][2 * u + 1]));
+          mx3 = fmax3(mx3, __uint_as_float(r[3][2 * u]), __uint_as_float(r[3][2 * u + 1]));
+        }
       }
+      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
       // Lazy rescale: a row moves its reference maximum only when the chunk's
-      // maximum exceeds it by more than 8 (a factor 2^8 in p).  The TMEM
-      // accesses below are warp-collective, so the decision is taken per warp;
-      // rows that keep their reference use alpha = 1.
+      // maximum exceeds it by more than 8 (a factor 2^8 in p); O and its row
+      // sums are rescaled after P is written (below).
       const float m_new = mx * kScaleLog2;
       const bool grow = m_new > m_ref + 8.0f;
-      if (__any_sync(0xffffffffu, grow)) {
-        const float alpha = grow ? fast_exp2(m_ref - m_new) : 1.0f;
-        if (c > 0) {
-          // The PV of chunk c-1 completed before S(c) was signalled.
-          uint32_t o[32];
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            tmem_ld32(tO + 32 * g, o);
-            tmem_ld_wait();
-#pragma unroll
-            for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
-            tmem_st32(tO + 32 * g, o);
-          }
-        }
-        if (grow) {
-          l *= alpha;
-          lr *= alpha;
-          m_ref = m_new;
-        }
+      const bool rescale_o = __any_sync(0xffffffffu, grow) && it > 0;
+      float alpha = 1.0f;
+      if (grow) {
+        alpha = fast_exp2(m_ref - m_new);   // 0 on the row's first kept chunk
+        l2.x *= alpha;
+        l2.y *= alpha;
+        l2b.x *= alpha;
+        l2b.y *= alpha;
+        m_ref = m_new;
       }
-      const float neg_m = -m_ref;
+      const float2 neg_m2 = make_float2(-m_ref, -m_ref);
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         const bool use = (g < 2) ? use0 : use1;
@@ -391,11 +479,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (use) {
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e]), kScaleLog2, neg_m));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e + 1]), kScaleLog2, neg_m));
-            l += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
-            lr += __uint_as_float(pk[e] << 16) + __uint_as_float(pk[e] & 0xFFFF0000u);
+            const float2 sv = make_float2(__uint_as_float(r[g][2 * e]), __uint_as_float(r[g][2 * e + 1]));
+            const float2 x = ffma2(sv, scale2, neg_m2);
+            const float2 pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            if (e & 1)
+              l2b = fadd2(l2b, pe);
+            else
+              l2 = fadd2(l2, pe);
+            pk[e] = pack_bf16x2(pe.x, pe.y);
           }
         } else {
 #pragma unroll
@@ -403,13 +494,38 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         tmem_st16(tS + 16 * g, pk);
       }
+      if (rescale_o) {
+        // This group's O and row sums hold its previous chunk (c - 2), whose
+        // PV completed before S(c) was signalled (S(c) is issued after it);
+        // they are rescaled before this chunk's PV is allowed to start.  The
+        // TMEM accesses are warp-collective, so the decision is per warp and
+        // rows that keep their reference use alpha = 1.
+        uint32_t o[32];
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          tmem_ld32(tO + 32 * g, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
+          tmem_st32(tO + 32 * g, o);
+        }
+        const uint32_t lv = tmem_ld1(tL);
+        tmem_ld_wait();
+        tmem_st1(tL, __float_as_uint(__uint_as_float(lv) * alpha));
+      }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_p);
     }
-    // Epilogue
+    const float l_sum = (l2.x + l2.y) + (l2b.x + l2b.y);
+    // Epilogue: the odd-chunk group posts its row statistics; the even-chunk
+    // group merges both partial results and writes the row.
     const int tok = row0 + row;
-    if (n_chunks == 0) {
+    if (par == 1) {
+      ctl->odd_m[row] = m_ref;
+      ctl->odd_l[row] = l_sum;
+      mbar_arrive(bar_merge);
+    } else if (n_chunks == 0) {
       if (tok < p.n) {
         float zero[64];
 #pragma unroll
@@ -418,24 +534,37 @@ __global__ void __launch_bounds__(kThreads, 2)
                   0.f);
         if (p.lse) p.lse[(size_t)h * p.n + tok] = -INFINITY;
       }
-    } else if (ok && warp_wait(bar_o, 0, abortf, p.err, 31)) {
+    } else if (ok && warp_wait(bar_o, 0, abortf, p.err, 31) &&
+               warp_wait(bar_merge, 0, abortf, p.err, 33)) {
       tc_fence_after();
-      uint32_t o[2][32];
-      tmem_ld32(tO, o[0]);
-      tmem_ld32(tO + 32, o[1]);
+      const bool two = n_chunks > 1;   // the odd group ran (its TMEM columns hold data)
+      const uint32_t lv0 = tmem_ld1(tL);
+      const uint32_t lv1 = two ? tmem_ld1(tL + 16) : 0u;
       tmem_ld_wait();
-      if (tok < p.n) {
-        float of[64];
+      const float m1v = two ? ctl->odd_m[row] : -INFINITY;
+      const float l1v = two ? ctl->odd_l[row] : 0.f;
+      const float m = fmaxf(m_ref, m1v);
+      const float a0 = fast_exp2(m_ref - m);    // 0 when this group never saw the row
+      const float a1 = two ? fast_exp2(m1v - m) : 0.f;
+      const float lr = fmaf(a1, __uint_as_float(lv1), a0 * __uint_as_float(lv0));
+      const float inv = 1.0f / lr;
+      OutT* dst = reinterpret_cast<OutT*>(p.out) + ((size_t)tok * p.heads + h) * kHeadDim;
+#pragma unroll
+      for (int hc = 0; hc < 2; ++hc) {
+        uint32_t oa[32], ob[32];
+        tmem_ld32(tO + 32 * hc, oa);
+        if (two) tmem_ld32(tO + 64 + 32 * hc, ob);
+        tmem_ld_wait();
+        float of[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
-          of[u] = __uint_as_float(o[0][u]);
-          of[32 + u] = __uint_as_float(o[1][u]);
+          of[u] = a0 * __uint_as_float(oa[u]);
+          if (two) of[u] = fmaf(a1, __uint_as_float(ob[u]), of[u]);
         }
-        const float inv = 1.0f / lr;
-        store_row(reinterpret_cast<OutT*>(p.out) + ((size_t)tok * p.heads + h) * kHeadDim, of,
-                  inv);
-        if (p.lse) p.lse[(size_t)h * p.n + tok] = (m_ref + __log2f(l)) * 0.6931471805599453f;
+        if (tok < p.n) store_half_row(dst + 32 * hc, of, inv);
       }
+      if (tok < p.n && p.lse)
+        p.lse[(size_t)h * p.n + tok] = (m + __log2f(a0 * l_sum + a1 * l1v)) * 0.6931471805599453f;
     }
   }
 
@@ -473,17 +602,17 @@ ress_status launch_attn(const Geometry& g, const void* q, const void* k, const v
   const size_t smem = attn_smem_bytes(g.nb);
   const dim3 grid((unsigned)(g.heads * p.tiles_per_head));
   if (out_f32) {
-    if (cudaFuncSetAttribute(block_sparse_attn_kernel<float>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return RESS_ERR_CUDA;
+    if (ress_status st_ = record_cuda(cudaFuncSetAttribute(block_sparse_attn_kernel<float>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+      return st_;
     block_sparse_attn_kernel<float><<<grid, kThreads, smem, st>>>(tq, tk, tv, p);
   } else {
-    if (cudaFuncSetAttribute(block_sparse_attn_kernel<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      return RESS_ERR_CUDA;
+    if (ress_status st_ = record_cuda(cudaFuncSetAttribute(block_sparse_attn_kernel<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+      return st_;
     block_sparse_attn_kernel<__nv_bfloat16><<<grid, kThreads, smem, st>>>(tq, tk, tv, p);
   }
-  return cudaGetLastError() == cudaSuccess ? RESS_OK : RESS_ERR_CUDA;
+  return record_cuda(cudaGetLastError());
 }
 
 }  // namespace ress

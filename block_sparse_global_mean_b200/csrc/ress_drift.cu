@@ -523,12 +523,12 @@ ress_status launch_drift(const Geometry& g, const void* q, const void* k, const 
   p.drift = drift;
   p.set_drift = set_drift;
   const size_t smem = drift_smem_bytes(g.nb);
-  if (cudaFuncSetAttribute(block_drift_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return RESS_ERR_CUDA;
+  if (ress_status st_ = record_cuda(cudaFuncSetAttribute(block_drift_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem)))
+    return st_;
   block_drift_kernel<<<(unsigned)(g.heads * p.tiles_per_head), kThreads, smem, st>>>(tq, tk, tv,
                                                                                      p);
-  return cudaGetLastError() == cudaSuccess ? RESS_OK : RESS_ERR_CUDA;
+  return record_cuda(cudaGetLastError());
 }
 
 }  // namespace ress

@@ -37,6 +37,10 @@ SelectLayout select_layout(const Geometry& g, bool with_v);
 // of 64 (d) x 1 (head) x `rows` (tokens), 128-byte swizzle.
 bool make_token_map(CUtensorMap* map, const void* base, const Geometry& g, int rows);
 
+// Records `err` as this thread's last CUDA error (for ress_last_cuda_error)
+// and returns RESS_ERR_CUDA, or RESS_OK for cudaSuccess.
+ress_status record_cuda(cudaError_t err);
+
 struct DeviceError;
 // Device address of the error flag on the current device (null on failure).
 DeviceError* device_error_ptr();

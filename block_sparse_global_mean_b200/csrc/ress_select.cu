@@ -305,11 +305,11 @@ ress_status launch_score(const ScoreArgs& a0, cudaStream_t st) {
   ScoreArgs a = a0;
   a.tiles_per_head = (a.nb + R - 1) / R;
   const size_t smem = score_smem_bytes<R>(a.nb_pad);
-  if (cudaFuncSetAttribute(score_topk_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem) != cudaSuccess)
-    return RESS_ERR_CUDA;
+  if (ress_status st_ = record_cuda(cudaFuncSetAttribute(score_topk_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem)))
+    return st_;
   score_topk_kernel<R><<<a.heads * a.tiles_per_head, 256, smem, st>>>(a);
-  return cudaGetLastError() == cudaSuccess ? RESS_OK : RESS_ERR_CUDA;
+  return record_cuda(cudaGetLastError());
 }
 
 }  // namespace
@@ -361,11 +361,11 @@ ress_status launch_select(const Geometry& g, const void* q, const void* k, const
     pool_kernel<float><<<grid, threads, red, st>>>(pa);
   else
     pool_kernel<__nv_bfloat16><<<grid, threads, red, st>>>(pa);
-  if (cudaGetLastError() != cudaSuccess) return RESS_ERR_CUDA;
+  if (ress_status st_ = record_cuda(cudaGetLastError())) return st_;
   if (with_v) {
     const int warps = g.heads * g.nb;
     contrast_kernel<<<(warps + 7) / 8, 256, 0, st>>>(vbar, contrast, g.heads, g.nb);
-    if (cudaGetLastError() != cudaSuccess) return RESS_ERR_CUDA;
+    if (ress_status st_ = record_cuda(cudaGetLastError())) return st_;
   }
   ScoreArgs sa{};
   sa.qbar = qbar;

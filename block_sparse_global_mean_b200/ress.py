@@ -63,6 +63,8 @@ lib.ress_block_drift.argtypes = [_SHAPE, _P, _P, _P, ctypes.c_int32, _P, _P, _P,
                                  ctypes.c_size_t, _P]
 lib.ress_select_blocks_noalloc.restype = ctypes.c_int
 lib.ress_select_blocks_noalloc.argtypes = [_SHAPE, _P, _P, _P, ctypes.c_int32, ctypes.c_float, _P, _P]
+lib.ress_last_cuda_error.restype = ctypes.c_char_p
+lib.ress_last_cuda_error.argtypes = []
 lib.ress_check_device_errors.restype = ctypes.c_int
 lib.ress_check_device_errors.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
 
@@ -71,6 +73,8 @@ class RessError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         msg = lib.ress_status_string(status).decode()
+        if status == RESS_ERR_CUDA:
+            msg += f" [{lib.ress_last_cuda_error().decode()}]"
         super().__init__(f"{where}: {msg} (status {status})")
 
 

@@ -207,6 +207,13 @@ ress_status ress_block_drift(const ress_shape* shape, const void* q, const void*
  */
 ress_status ress_check_device_errors(void* stream, int32_t* detail);
 
+/*
+ * Name and message of the last CUDA error behind a RESS_ERR_CUDA returned to
+ * the calling host thread ("" if none).  The string stays valid until the
+ * thread's next library call.
+ */
+const char* ress_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif
