@@ -10,11 +10,11 @@
 //
 // Warp roles (320 threads, one CTA per SM):
 //   warp 0     TMA producer: Q tile once, then K/V sub-blocks of each chunk
-//              into a 4-stage ring (128-byte swizzle).
+//              into a 5-stage ring (128-byte swizzle).
 //   warp 1     TMEM owner and MMA issuer: S = Q K^T (M=128, N=128, K=64) into
-//              one of two TMEM buffers, so S of chunk c+1 is computed while the
-//              softmax warps work on chunk c; then O += P V (M=128, N=64,
-//              K=128) with P read from TMEM.
+//              one of three TMEM buffers, so the S of a softmax group's next
+//              chunk is ready when it finishes the current one; then
+//              O += P V (M=128, N=64, K=128) with P read from TMEM.
 //   warps 2-9  softmax, one query row per thread, in two groups: warps 2-5
 //              take the even chunks and warps 6-9 the odd ones, each group with
 //              its own running maximum, sums and O accumulator in TMEM (a
@@ -23,9 +23,8 @@
 //              S is read from TMEM, the online softmax runs in the log2 domain
 //              with a lazy rescale of O (only when the running maximum grows
 //              by more than 2^8), and P goes back to TMEM as bf16 over the
-//              first 64 columns of S; epilogue O / sum(P) and lse.
-//              The row sums of the bf16 P come from one more MMA, P times a
-//              16-column tile of ones (N=16), accumulated next to O.
+//              first 64 columns of S; epilogue O / sum(P) and lse, where
+//              sum(P) adds the same bf16-rounded values that enter P V.
 //
 // Every mbarrier wait is bounded; on timeout the CTA raises the device error,
 // drains its copies and MMAs in flight, frees TMEM and exits.
@@ -37,18 +36,16 @@ namespace ress {
 namespace {
 
 constexpr int kRows = 128;
-constexpr int kStages = 4;
+constexpr int kStages = 5;
+constexpr int kSBufs = 3;
 constexpr int kThreads = 320;
 constexpr uint32_t kQBytes = 128 * 128;            // 128 rows x 64 bf16
 constexpr uint32_t kSubBytes = 64 * 128;           // 64 keys x 64 bf16
 constexpr uint32_t kStageBytes = 4 * kSubBytes;    // K sub0, K sub1, V sub0, V sub1
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;                      // S buffers at 0 and 128 (128 fp32 columns each;
+constexpr uint32_t kColS = 0;                      // S buffers at 0, 128, 256 (128 fp32 columns each;
                                                    // P as bf16 in the first 64 columns of its buffer)
-constexpr uint32_t kColO = 256;                    // O of the even / odd chunks: 2 x 64 fp32 columns
-constexpr uint32_t kColL = 384;                    // row sums of the bf16 P (P times a ones tile),
-                                                   // even / odd chunks: 2 x 16 columns
-constexpr uint32_t kOnesBytes = 16 * 128;          // 16 x 64 bf16 ones, K-major, 128-byte swizzle
+constexpr uint32_t kColO = 384;                    // O of the even / odd chunks: 2 x 64 fp32 columns
 
 struct AttnParams {
   DeviceError* err;
@@ -67,10 +64,11 @@ struct __align__(8) Ctl {
   uint64_t q_full;
   uint64_t kv_full[kStages];
   uint64_t kv_empty[kStages];
-  uint64_t s_full[2];   // S buffer b holds S of chunk c (c % 2 == b)
-  uint64_t p_full[2];   // P of chunk c written into S buffer c % 2
+  uint64_t s_full[kSBufs];   // S buffer b holds S of chunk c (c % 3 == b)
+  uint64_t p_full[kSBufs];   // P of chunk c written into S buffer c % 3
+  uint64_t o_done[2];        // PV of a chunk of group g (c % 2 == g) completed
   uint64_t o_full;
-  uint64_t merge;       // the odd-chunk group posted its row statistics
+  uint64_t merge;            // the odd-chunk group posted its row statistics
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort_flag;
@@ -78,12 +76,13 @@ struct __align__(8) Ctl {
   int pad;
   float odd_m[kRows];   // odd-chunk group: reference maximum (log2 domain) per row
   float odd_l[kRows];   // odd-chunk group: float32 probability sum per row
+  float odd_lr[kRows];  // odd-chunk group: sum of the bf16-rounded probabilities
 };
 
 __host__ __device__ inline int words_for(int nb) { return (nb + 31) >> 5; }
 
 size_t attn_smem_bytes(int nb) {
-  return 1024 + kQBytes + kStages * kStageBytes + kOnesBytes + sizeof(Ctl) +
+  return 1024 + kQBytes + kStages * kStageBytes + sizeof(Ctl) +
          sizeof(uint32_t) * (2 * (size_t)words_for(nb) + (size_t)nb);
 }
 
@@ -184,8 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                              ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + kQBytes;
-  uint8_t* sOnes = sKV + kStages * kStageBytes;
-  Ctl* ctl = reinterpret_cast<Ctl*>(sOnes + kOnesBytes);
+  Ctl* ctl = reinterpret_cast<Ctl*>(sKV + kStages * kStageBytes);
   const int W = words_for(p.nb);
   uint32_t* bmA = reinterpret_cast<uint32_t*>(ctl + 1);
   uint32_t* bmB = bmA + W;
@@ -202,6 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bar_q = smem_addr(&ctl->q_full);
   const uint32_t bar_s0 = smem_addr(&ctl->s_full[0]);
   const uint32_t bar_p0 = smem_addr(&ctl->p_full[0]);
+  const uint32_t bar_od0 = smem_addr(&ctl->o_done[0]);
   const uint32_t bar_o = smem_addr(&ctl->o_full);
   const uint32_t bar_merge = smem_addr(&ctl->merge);
   const uint32_t bar_done = smem_addr(&ctl->mma_done);
@@ -213,10 +212,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_addr(&ctl->kv_full[s]), 1);
       mbar_init(smem_addr(&ctl->kv_empty[s]), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kSBufs; ++b) {
       mbar_init(bar_s0 + 8 * b, 1);
       mbar_init(bar_p0 + 8 * b, 128);
     }
+    mbar_init(bar_od0, 1);
+    mbar_init(bar_od0 + 8, 1);
     mbar_init(bar_o, 1);
     mbar_init(bar_merge, 128);
     mbar_init(bar_done, 1);
@@ -228,10 +229,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   for (int w = threadIdx.x; w < 2 * W; w += kThreads) bmA[w] = 0u;
-  // bf16 ones: the B operand of the MMA that sums each row of P.
-  for (int w = threadIdx.x; w < (int)(kOnesBytes / 4); w += kThreads)
-    reinterpret_cast<uint32_t*>(sOnes)[w] = 0x3F803F80u;
-  fence_proxy_async_smem();
   __syncthreads();
 
   // Kept sets of the tile's query blocks as bitmaps (duplicates collapse,
@@ -327,11 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (n_chunks > 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idPV = idesc_bf16_f32(128, 64, true);
-      constexpr uint32_t idL = idesc_bf16_f32(128, 16, false);
       const uint32_t tS = tmem + kColS;
       const uint32_t tO = tmem + kColO;
-      const uint32_t tL = tmem + kColL;
-      const uint64_t dones = smem_desc_sw128(smem_addr(sOnes), 16, 1024);
       const uint64_t dq = smem_desc_sw128(smem_addr(sQ), 16, 1024);
       // Stage s: K at +s*kStageBytes, V at +2*kSubBytes; one 16-key step of V
       // is 2048 bytes (128 units of 16 bytes in the descriptor's address field).
@@ -341,16 +335,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = warp_wait(bar_q, 0, abortf, p.err, 20);
       auto issue_s = [&](int c) -> bool {
         const int s = c % kStages;
+        const int b = c % kSBufs;
         if (!warp_wait(smem_addr(&ctl->kv_full[s]), (c / kStages) & 1, abortf, p.err, 22))
           return false;
         tc_fence_after();
         const uint64_t dk = dk0 + (uint64_t)s * kStageDesc;
-        const uint32_t tSb = tS + 128u * (uint32_t)(c & 1);
+        const uint32_t tSb = tS + 128u * (uint32_t)b;
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ss(tSb, dq + (uint64_t)(kk * 2), dk + (uint64_t)(kk * 2), idS, kk > 0 ? 1u : 0u);
-          mma_commit(bar_s0 + 8u * (uint32_t)(c & 1));
+          mma_commit(bar_s0 + 8u * (uint32_t)b);
         }
         __syncwarp();
         return true;
@@ -358,33 +353,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto issue_pv = [&](int c) {
         const int sp = c % kStages;
         const uint64_t dv = dv0 + (uint64_t)sp * kStageDesc;
-        const uint32_t par = (uint32_t)(c & 1);
-        const uint32_t tP = tS + 128u * par;
-        const uint32_t tOp = tO + 64u * par;
-        const uint32_t tLp = tL + 16u * par;
+        const uint32_t tP = tS + 128u * (uint32_t)(c % kSBufs);
+        const uint32_t tOp = tO + 64u * (uint32_t)(c & 1);
         const uint32_t acc0 = c > 1 ? 1u : 0u;
         if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tOp, tP + kk * 8, dv + (uint64_t)(kk * 128), idPV, kk > 0 ? 1u : acc0);
-          // Row sums of the same bf16 P: every 16-key slice of the ones tile is 1.
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk) mma_ts(tLp, tP + kk * 8, dones, idL, kk > 0 ? 1u : acc0);
           mma_commit(smem_addr(&ctl->kv_empty[sp]));
+          mma_commit(bar_od0 + 8u * (uint32_t)(c & 1));
         }
         __syncwarp();
       };
-      if (ok) ok = issue_s(0);
+      for (int c = 0; ok && c < n_chunks && c < kSBufs; ++c) ok = issue_s(c);
       for (int c = 0; ok && c < n_chunks; ++c) {
-        // S(c+1) goes to the other buffer, which holds P(c-1): PV(c-1) was
-        // issued before it, and the tensor core runs the MMAs in issue order.
-        if (c + 1 < n_chunks && !(ok = issue_s(c + 1))) break;
-        if (!warp_wait(bar_p0 + 8u * (uint32_t)(c & 1), (c >> 1) & 1, abortf, p.err, 21)) {
+        if (!warp_wait(bar_p0 + 8u * (uint32_t)(c % kSBufs), (c / kSBufs) & 1, abortf, p.err, 21)) {
           ok = false;
           break;
         }
         tc_fence_after();
         issue_pv(c);
+        // S(c+3) reuses the buffer of P(c); the tensor core runs the MMAs in
+        // issue order, so PV(c) has read P(c) before S(c+3) overwrites it.
+        if (c + kSBufs < n_chunks && !(ok = issue_s(c + kSBufs))) break;
       }
       if (elect_one()) {
         if (ok) mma_commit(bar_o);
@@ -401,19 +392,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int row = quad * 32 + lane;
     const int half = row >> 6;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t tS = tmem + kColS + lane_off + 128u * (uint32_t)par;
+    const uint32_t tS0 = tmem + kColS + lane_off;
     const uint32_t tO = tmem + kColO + lane_off + 64u * (uint32_t)par;
-    const uint32_t tL = tmem + kColL + lane_off + 16u * (uint32_t)par;
-    const uint32_t bar_s = bar_s0 + 8u * (uint32_t)par;
-    const uint32_t bar_p = bar_p0 + 8u * (uint32_t)par;
+    const uint32_t bar_od = bar_od0 + 8u * (uint32_t)par;
     const float kScaleLog2 = 1.4426950408889634f * 0.125f;   // log2(e) / sqrt(64)
     const float2 scale2 = make_float2(kScaleLog2, kScaleLog2);
     float m_ref = -INFINITY;
     float2 l2 = make_float2(0.f, 0.f);   // float32 probability sums (for lse)
     float2 l2b = make_float2(0.f, 0.f);
+    float2 lr2 = make_float2(0.f, 0.f);  // sums of the bf16-rounded probabilities (normaliser)
     bool ok = true;
     for (int c = par, it = 0; c < n_chunks; c += 2, ++it) {
-      if (!warp_wait(bar_s, it & 1, abortf, p.err, 30)) {
+      const int b = c % kSBufs;
+      const uint32_t tS = tS0 + 128u * (uint32_t)b;
+      const uint32_t bar_p = bar_p0 + 8u * (uint32_t)b;
+      if (!warp_wait(bar_s0 + 8u * (uint32_t)b, (c / kSBufs) & 1, abortf, p.err, 30)) {
         ok = false;
         break;
       }
@@ -469,6 +462,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         l2.y *= alpha;
         l2b.x *= alpha;
         l2b.y *= alpha;
+        lr2.x *= alpha;
+        lr2.y *= alpha;
         m_ref = m_new;
       }
       const float2 neg_m2 = make_float2(-m_ref, -m_ref);
@@ -487,6 +482,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             else
               l2 = fadd2(l2, pe);
             pk[e] = pack_bf16x2(pe.x, pe.y);
+            lr2 = fadd2(lr2, make_float2(__uint_as_float(pk[e] << 16),
+                                         __uint_as_float(pk[e] & 0xFFFF0000u)));
           }
         } else {
 #pragma unroll
@@ -495,11 +492,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st16(tS + 16 * g, pk);
       }
       if (rescale_o) {
-        // This group's O and row sums hold its previous chunk (c - 2), whose
-        // PV completed before S(c) was signalled (S(c) is issued after it);
-        // they are rescaled before this chunk's PV is allowed to start.  The
+        // This group's O holds its previous chunk (c - 2) once that PV has
+        // completed (its commit is this group's o_done phase it - 1; the PV
+        // before it completed before S(c) was signalled, so the parity is
+        // unambiguous).  O is rescaled before this chunk's PV may start.  The
         // TMEM accesses are warp-collective, so the decision is per warp and
         // rows that keep their reference use alpha = 1.
+        if (!warp_wait(bar_od, (it - 1) & 1, abortf, p.err, 32)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
         uint32_t o[32];
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
@@ -509,21 +512,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
           tmem_st32(tO + 32 * g, o);
         }
-        const uint32_t lv = tmem_ld1(tL);
-        tmem_ld_wait();
-        tmem_st1(tL, __float_as_uint(__uint_as_float(lv) * alpha));
       }
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(bar_p);
     }
     const float l_sum = (l2.x + l2.y) + (l2b.x + l2b.y);
+    const float lr_sum = lr2.x + lr2.y;
     // Epilogue: the odd-chunk group posts its row statistics; the even-chunk
     // group merges both partial results and writes the row.
     const int tok = row0 + row;
     if (par == 1) {
       ctl->odd_m[row] = m_ref;
       ctl->odd_l[row] = l_sum;
+      ctl->odd_lr[row] = lr_sum;
       mbar_arrive(bar_merge);
     } else if (n_chunks == 0) {
       if (tok < p.n) {
@@ -538,15 +540,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                warp_wait(bar_merge, 0, abortf, p.err, 33)) {
       tc_fence_after();
       const bool two = n_chunks > 1;   // the odd group ran (its TMEM columns hold data)
-      const uint32_t lv0 = tmem_ld1(tL);
-      const uint32_t lv1 = two ? tmem_ld1(tL + 16) : 0u;
-      tmem_ld_wait();
       const float m1v = two ? ctl->odd_m[row] : -INFINITY;
       const float l1v = two ? ctl->odd_l[row] : 0.f;
+      const float lr1 = two ? ctl->odd_lr[row] : 0.f;
       const float m = fmaxf(m_ref, m1v);
       const float a0 = fast_exp2(m_ref - m);    // 0 when this group never saw the row
       const float a1 = two ? fast_exp2(m1v - m) : 0.f;
-      const float lr = fmaf(a1, __uint_as_float(lv1), a0 * __uint_as_float(lv0));
+      const float lr = fmaf(a1, lr1, a0 * lr_sum);
       const float inv = 1.0f / lr;
       OutT* dst = reinterpret_cast<OutT*>(p.out) + ((size_t)tok * p.heads + h) * kHeadDim;
 #pragma unroll
@@ -600,6 +600,7 @@ ress_status launch_attn(const Geometry& g, const void* q, const void* k, const v
   p.out = out;
   p.lse = lse;
   const size_t smem = attn_smem_bytes(g.nb);
+  if (smem > 227 * 1024) return RESS_ERR_UNSUPPORTED;   // kept-block lists no longer fit
   const dim3 grid((unsigned)(g.heads * p.tiles_per_head));
   if (out_f32) {
     if (ress_status st_ = record_cuda(cudaFuncSetAttribute(block_sparse_attn_kernel<float>,

@@ -523,6 +523,7 @@ ress_status launch_drift(const Geometry& g, const void* q, const void* k, const 
   p.drift = drift;
   p.set_drift = set_drift;
   const size_t smem = drift_smem_bytes(g.nb);
+  if (smem > 227 * 1024) return RESS_ERR_UNSUPPORTED;   // block lists no longer fit
   if (ress_status st_ = record_cuda(cudaFuncSetAttribute(block_drift_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem)))
     return st_;

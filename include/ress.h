@@ -163,6 +163,8 @@ size_t ress_attn_workspace_bytes(const ress_shape* shape);
  *   out        [N][H][64] of `out_dtype` (RESS_BF16 or RESS_F32, independent
  *              of the input dtype).
  *   lse        [H][N] float32, or NULL.
+ *   Supported sizes: nb <= 10,000 (the kept-block lists live in shared
+ *   memory); larger grids return RESS_ERR_UNSUPPORTED.
  *   The contractions run on bf16 operands with float32 accumulation; the
  *   probabilities enter P V as bf16 and the row normaliser is the sum of those
  *   same bf16 values, so each output row is a convex combination of kept
