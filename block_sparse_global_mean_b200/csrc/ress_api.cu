@@ -259,4 +259,9 @@ ress_status ress_check_device_errors(void* stream, int32_t* detail) {
 
 const char* ress_last_cuda_error(void) { return g_last_cuda_error; }
 
+ress_status ress_test_exp2(const float* x, float* y, int32_t n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return RESS_ERR_INVALID_ARG;
+  return launch_exp2_poly_test(x, y, n, static_cast<cudaStream_t>(stream));
+}
+
 }  // extern "C"

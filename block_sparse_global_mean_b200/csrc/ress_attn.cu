@@ -75,7 +75,6 @@ struct __align__(8) Ctl {
   int n_entries;
   int pad;
   float odd_m[kRows];   // odd-chunk group: reference maximum (log2 domain) per row
-  float odd_l[kRows];   // odd-chunk group: float32 probability sum per row
   float odd_lr[kRows];  // odd-chunk group: sum of the bf16-rounded probabilities
 };
 
@@ -398,9 +397,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float kScaleLog2 = 1.4426950408889634f * 0.125f;   // log2(e) / sqrt(64)
     const float2 scale2 = make_float2(kScaleLog2, kScaleLog2);
     float m_ref = -INFINITY;
-    float2 l2 = make_float2(0.f, 0.f);   // float32 probability sums (for lse)
-    float2 l2b = make_float2(0.f, 0.f);
-    float2 lr2 = make_float2(0.f, 0.f);  // sums of the bf16-rounded probabilities (normaliser)
+    // Sums of the bf16-rounded probabilities that enter P V: the normaliser
+    // of O and the sum behind lse (two independent accumulators per row).
+    float lr_lo = 0.f, lr_hi = 0.f;
     bool ok = true;
     for (int c = par, it = 0; c < n_chunks; c += 2, ++it) {
       const int b = c % kSBufs;
@@ -458,12 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       float alpha = 1.0f;
       if (grow) {
         alpha = fast_exp2(m_ref - m_new);   // 0 on the row's first kept chunk
-        l2.x *= alpha;
-        l2.y *= alpha;
-        l2b.x *= alpha;
-        l2b.y *= alpha;
-        lr2.x *= alpha;
-        lr2.y *= alpha;
+        lr_lo *= alpha;
+        lr_hi *= alpha;
         m_ref = m_new;
       }
       const float2 neg_m2 = make_float2(-m_ref, -m_ref);
@@ -476,14 +471,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 16; ++e) {
             const float2 sv = make_float2(__uint_as_float(r[g][2 * e]), __uint_as_float(r[g][2 * e + 1]));
             const float2 x = ffma2(sv, scale2, neg_m2);
-            const float2 pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
-            if (e & 1)
-              l2b = fadd2(l2b, pe);
-            else
-              l2 = fadd2(l2, pe);
+            // One pair in eight goes to the FMA pipe, the rest to MUFU.
+            const float2 pe = ((e & 7) == 7) ? exp2_poly2(x)
+                                             : make_float2(fast_exp2(x.x), fast_exp2(x.y));
             pk[e] = pack_bf16x2(pe.x, pe.y);
-            lr2 = fadd2(lr2, make_float2(__uint_as_float(pk[e] << 16),
-                                         __uint_as_float(pk[e] & 0xFFFF0000u)));
+            lr_lo = add_bf16_lo(pk[e], lr_lo);
+            lr_hi = add_bf16_hi(pk[e], lr_hi);
           }
         } else {
 #pragma unroll
@@ -517,14 +510,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive(bar_p);
     }
-    const float l_sum = (l2.x + l2.y) + (l2b.x + l2b.y);
-    const float lr_sum = lr2.x + lr2.y;
+    const float lr_sum = lr_lo + lr_hi;
     // Epilogue: the odd-chunk group posts its row statistics; the even-chunk
     // group merges both partial results and writes the row.
     const int tok = row0 + row;
     if (par == 1) {
       ctl->odd_m[row] = m_ref;
-      ctl->odd_l[row] = l_sum;
       ctl->odd_lr[row] = lr_sum;
       mbar_arrive(bar_merge);
     } else if (n_chunks == 0) {
@@ -541,7 +532,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const bool two = n_chunks > 1;   // the odd group ran (its TMEM columns hold data)
       const float m1v = two ? ctl->odd_m[row] : -INFINITY;
-      const float l1v = two ? ctl->odd_l[row] : 0.f;
       const float lr1 = two ? ctl->odd_lr[row] : 0.f;
       const float m = fmaxf(m_ref, m1v);
       const float a0 = fast_exp2(m_ref - m);    // 0 when this group never saw the row
@@ -564,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tok < p.n) store_half_row(dst + 32 * hc, of, inv);
       }
       if (tok < p.n && p.lse)
-        p.lse[(size_t)h * p.n + tok] = (m + __log2f(a0 * l_sum + a1 * l1v)) * 0.6931471805599453f;
+        p.lse[(size_t)h * p.n + tok] = (m + __log2f(lr)) * 0.6931471805599453f;
     }
   }
 
@@ -576,7 +566,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+__global__ void exp2_poly_test_kernel(const float* __restrict__ x, float* __restrict__ y, int n) {
+  const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+  if (i + 1 < n) {
+    const float2 r = exp2_poly2(make_float2(x[i], x[i + 1]));
+    y[i] = r.x;
+    y[i + 1] = r.y;
+  } else if (i < n) {
+    y[i] = exp2_poly2(make_float2(x[i], 0.f)).x;
+  }
+}
+
 }  // namespace
+
+ress_status launch_exp2_poly_test(const float* x, float* y, int n, cudaStream_t st) {
+  if (n <= 0) return RESS_OK;
+  const int pairs = (n + 1) / 2;
+  exp2_poly_test_kernel<<<(pairs + 255) / 256, 256, 0, st>>>(x, y, n);
+  return record_cuda(cudaGetLastError());
+}
 
 bool make_token_map(CUtensorMap* map, const void* base, const Geometry& g, int rows);
 

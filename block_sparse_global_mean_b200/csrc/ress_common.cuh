@@ -292,6 +292,43 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return d;
 }
 
+// 2^x for a pair of float32 values on the FMA and integer pipes (no MUFU):
+// range reduction 2^x = 2^n * 2^f with n = round(x) (the 1.5 * 2^23 shifter
+// rounds to nearest) and f = x - n in [-1/2, 1/2], then a degree-3 polynomial
+// for 2^f whose coefficients come from fit_exp2_poly.py (Lawson's minimax
+// fit; max relative error 7.5e-5 in float32, below bf16's 2^-9), and n is
+// added to the exponent field.  Inputs are clamped to >= -126 so the result
+// stays a (tiny) finite value; callers pass x <= 8.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kShift = 12582912.0f;   // 1.5 * 2^23
+  x.x = fmaxf(x.x, -126.0f);
+  x.y = fmaxf(x.y, -126.0f);
+  const float2 t = fadd2(x, make_float2(kShift, kShift));
+  const float2 n = fadd2(t, make_float2(-kShift, -kShift));
+  const float2 f = ffma2(n, make_float2(-1.0f, -1.0f), x);
+  float2 q = ffma2(make_float2(0.0551714338f, 0.0551714338f), f,
+                   make_float2(0.242610812f, 0.242610812f));
+  q = ffma2(q, f, make_float2(0.693260968f, 0.693260968f));
+  q = ffma2(q, f, make_float2(0.999928117f, 0.999928117f));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
+// acc + (bf16 in the low / high half of `pk`), accumulated in float32
+// (sm_100 mixed-precision add).
+__device__ __forceinline__ float add_bf16_lo(uint32_t pk, float acc) {
+  float r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.bf16 %0, l, %2;\n\t}"
+      : "=f"(r) : "r"(pk), "f"(acc));
+  return r;
+}
+__device__ __forceinline__ float add_bf16_hi(uint32_t pk, float acc) {
+  float r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tadd.rn.f32.bf16 %0, h, %2;\n\t}"
+      : "=f"(r) : "r"(pk), "f"(acc));
+  return r;
+}
+
 // Makes this thread's generic-proxy shared-memory writes visible to the
 // async proxy (TMA, tcgen05.mma operand reads).
 __device__ __forceinline__ void fence_proxy_async_smem() {

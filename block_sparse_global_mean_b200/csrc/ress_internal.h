@@ -54,6 +54,7 @@ ress_status launch_attn(const Geometry& g, const void* q, const void* k, const v
 ress_status launch_drift(const Geometry& g, const void* q, const void* k, const void* v,
                          int budget, const int32_t* idx, const float* lse, float* drift,
                          float* set_drift, cudaStream_t st);
+ress_status launch_exp2_poly_test(const float* x, float* y, int n, cudaStream_t st);
 ress_status launch_cast_bf16(const float* src, __nv_bfloat16* dst, size_t count, cudaStream_t st);
 
 }  // namespace ress

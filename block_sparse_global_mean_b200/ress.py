@@ -65,6 +65,8 @@ lib.ress_select_blocks_noalloc.restype = ctypes.c_int
 lib.ress_select_blocks_noalloc.argtypes = [_SHAPE, _P, _P, _P, ctypes.c_int32, ctypes.c_float, _P, _P]
 lib.ress_last_cuda_error.restype = ctypes.c_char_p
 lib.ress_last_cuda_error.argtypes = []
+lib.ress_test_exp2.restype = ctypes.c_int
+lib.ress_test_exp2.argtypes = [_P, _P, ctypes.c_int32, _P]
 lib.ress_check_device_errors.restype = ctypes.c_int
 lib.ress_check_device_errors.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
 

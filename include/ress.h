@@ -168,7 +168,8 @@ size_t ress_attn_workspace_bytes(const ress_shape* shape);
  *   The contractions run on bf16 operands with float32 accumulation; the
  *   probabilities enter P V as bf16 and the row normaliser is the sum of those
  *   same bf16 values, so each output row is a convex combination of kept
- *   values.  lse uses the float32 probabilities.
+ *   values, and lse is the log of that same sum (it differs from the float32
+ *   log-sum-exp by at most ln(1 + 2^-9) < 2e-3).
  */
 ress_status ress_block_sparse_attn(const ress_shape* shape, const void* q, const void* k,
                                    const void* v, int32_t budget, const int32_t* idx,
@@ -215,6 +216,15 @@ ress_status ress_check_device_errors(void* stream, int32_t* detail);
  * thread's next library call.
  */
 const char* ress_last_cuda_error(void);
+
+/*
+ * Test hook: y[i] = 2^x[i] computed by the polynomial exponential that the
+ * attention kernel uses for part of its probabilities (range reduction plus
+ * a degree-3 minimax polynomial on the FMA pipe; relative error <= 1e-4 for
+ * -100 <= x <= 8, a finite value below 2^-99 under that).  x and y are device
+ * arrays of n float32.
+ */
+ress_status ress_test_exp2(const float* x, float* y, int32_t n, void* stream);
 
 #ifdef __cplusplus
 }
