@@ -256,28 +256,35 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_chunks = (p.block == 64) ? (n_entries + 1) / 2 : n_entries;
 
   if (warp == 0) {
-    if (lane == 0 && n_chunks > 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(bar_q, kQBytes);
-      tma_load_3d(smem_addr(sQ), &tm_q, bar_q, 0, h, row0);
+    // TMA producer: the whole warp follows, one elected lane issues.
+    if (n_chunks > 0) {
+      if (elect_one()) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        mbar_arrive_expect_tx(bar_q, kQBytes);
+        tma_load_3d(smem_addr(sQ), &tm_q, bar_q, 0, h, row0);
+      }
+      __syncwarp();
       int issued = 0;
       for (int c = 0; c < n_chunks; ++c) {
         const int s = c % kStages;
         if (c >= kStages &&
-            !mbar_wait(smem_addr(&ctl->kv_empty[s]), ((c / kStages) - 1) & 1, abortf, p.err, 40))
+            !warp_wait(smem_addr(&ctl->kv_empty[s]), ((c / kStages) - 1) & 1, abortf, p.err, 40))
           break;
         int t0, t1;
         uint32_t j0, j1, m0, m1;
         chunk_info(list, n_entries, p.block, c, t0, t1, j0, j1, m0, m1);
-        uint8_t* st = sKV + s * kStageBytes;
+        const uint32_t st = smem_addr(sKV) + (uint32_t)s * kStageBytes;
         const uint32_t bar = smem_addr(&ctl->kv_full[s]);
-        mbar_arrive_expect_tx(bar, kStageBytes);
-        tma_load_3d(smem_addr(st), &tm_k, bar, 0, h, t0);
-        tma_load_3d(smem_addr(st + kSubBytes), &tm_k, bar, 0, h, t1);
-        tma_load_3d(smem_addr(st + 2 * kSubBytes), &tm_v, bar, 0, h, t0);
-        tma_load_3d(smem_addr(st + 3 * kSubBytes), &tm_v, bar, 0, h, t1);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar, kStageBytes);
+          tma_load_3d(st, &tm_k, bar, 0, h, t0);
+          tma_load_3d(st + kSubBytes, &tm_k, bar, 0, h, t1);
+          tma_load_3d(st + 2 * kSubBytes, &tm_v, bar, 0, h, t0);
+          tma_load_3d(st + 3 * kSubBytes, &tm_v, bar, 0, h, t1);
+        }
+        __syncwarp();
         issued = c + 1;
       }
       for (int c = issued > kStages ? issued - kStages : 0; c < issued; ++c)
@@ -286,49 +293,58 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0 && n_chunks > 0) {
+    // MMA issuer: the whole warp follows, one elected lane issues.
+    if (n_chunks > 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idPV = idesc_bf16_f32(128, 64, true);
       const uint32_t tS = tmem + kColS;
       const uint64_t dq = smem_desc_sw128(smem_addr(sQ), 16, 1024);
-      bool ok = mbar_wait(bar_q, 0, abortf, p.err, 50);
+      const uint64_t dk0 = smem_desc_sw128(smem_addr(sKV), 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(smem_addr(sKV) + 2 * kSubBytes, 16384, 1024);
+      constexpr uint64_t kStageDesc = kStageBytes >> 4;
+      constexpr uint64_t kSubDesc = kSubBytes >> 4;
+      bool ok = warp_wait(bar_q, 0, abortf, p.err, 50);
       for (int c = 0; ok && c < n_chunks; ++c) {
         const int s = c % kStages;
-        if (!mbar_wait(smem_addr(&ctl->kv_full[s]), (c / kStages) & 1, abortf, p.err, 51)) break;
+        if (!warp_wait(smem_addr(&ctl->kv_full[s]), (c / kStages) & 1, abortf, p.err, 51)) break;
         tc_fence_after();
-        const uint64_t dk = smem_desc_sw128(smem_addr(sKV + s * kStageBytes), 16, 1024);
+        const uint64_t dk = dk0 + (uint64_t)s * kStageDesc;
+        const uint64_t dv = dv0 + (uint64_t)s * kStageDesc;
+        if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ss(tS, dq + (uint64_t)(kk * 2), dk + (uint64_t)(kk * 2), idS, kk > 0 ? 1u : 0u);
-        mma_commit(bar_s);
-        if (!mbar_wait(bar_p, c & 1, abortf, p.err, 52)) break;
-        if (c > 0 && !mbar_wait(bar_cf, (c - 1) & 1, abortf, p.err, 53)) break;
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tS, dq + (uint64_t)(kk * 2), dk + (uint64_t)(kk * 2), idS, kk > 0 ? 1u : 0u);
+          mma_commit(bar_s);
+        }
+        __syncwarp();
+        if (!warp_wait(bar_p, c & 1, abortf, p.err, 52)) break;
+        if (c > 0 && !warp_wait(bar_cf, (c - 1) & 1, abortf, p.err, 53)) break;
         tc_fence_after();
-        const uint32_t vaddr = smem_addr(sKV + s * kStageBytes + 2 * kSubBytes);
-        if (p.block == 64) {
+        if (elect_one()) {
+          if (p.block == 64) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            mma_ts(tmem + kColC0, tS + kk * 8,
-                   smem_desc_sw128(vaddr + kk * 2048, 16384, 1024), idPV, kk > 0 ? 1u : 0u);
-            mma_ts(tmem + kColC1, tS + 32 + kk * 8,
-                   smem_desc_sw128(vaddr + kSubBytes + kk * 2048, 16384, 1024), idPV,
-                   kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {
+              mma_ts(tmem + kColC0, tS + kk * 8, dv + (uint64_t)(kk * 128), idPV, kk > 0 ? 1u : 0u);
+              mma_ts(tmem + kColC1, tS + 32 + kk * 8, dv + kSubDesc + (uint64_t)(kk * 128), idPV,
+                     kk > 0 ? 1u : 0u);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk)
+              mma_ts(tmem + kColC0, tS + kk * 8, dv + (uint64_t)(kk * 128), idPV, kk > 0 ? 1u : 0u);
           }
-        } else {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + kColC0, tS + kk * 8, smem_desc_sw128(vaddr + kk * 2048, 16384, 1024),
-                   idPV, kk > 0 ? 1u : 0u);
+            mma_ts(tmem + kColT, tS + kk * 8, dv + (uint64_t)(kk * 128), idPV,
+                   (c > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(bar_c);
+          mma_commit(smem_addr(&ctl->kv_empty[s]));
+          if (c == n_chunks - 1) mma_commit(bar_t);
         }
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + kColT, tS + kk * 8, smem_desc_sw128(vaddr + kk * 2048, 16384, 1024), idPV,
-                 (c > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(bar_c);
-        mma_commit(smem_addr(&ctl->kv_empty[s]));
-        if (c == n_chunks - 1) mma_commit(bar_t);
+        __syncwarp();
       }
-      mma_commit(bar_done);
+      if (elect_one()) mma_commit(bar_done);
+      __syncwarp();
       mbar_wait_drain(bar_done, 0, p.err, 54);
     }
     __syncwarp();

@@ -5,9 +5,11 @@
 //   contrast_kernel    c[h][j] = ||Vbar_j - Vbar_{j-1}||_2, c[h][0] = 0.
 //   score_topk_kernel  per (head, R query blocks): pooled logits for every key
 //                      block into shared memory (fp32 FMA), optional softmax +
-//                      contrast, then an exact radix select per row (one warp
-//                      per row) that keeps `budget` blocks, ties to the lower
-//                      index, written in ascending order.
+//                      contrast, then an exact selection per row (one warp per
+//                      row: a value-linear histogram finds the threshold bin,
+//                      whose few values are ranked exactly) that keeps
+//                      `budget` blocks, ties to the lower index, written in
+//                      ascending order.
 //
 // Sources: ReSS (thelatestinai.com) Table S5, SpargeAttn row - selection by
 // pooled query/key inner products; VASC (paperlayer.ai) 4.1 - pooled relevance
@@ -210,6 +212,145 @@ __device__ __forceinline__ void warp_topk_row(const float* row, int nb, int budg
   }
 }
 
+constexpr int kBins = 512;        // linear histogram bins over [row min, row max]
+constexpr int kMaxCand = 64;      // candidates resolved exactly in the threshold bin
+constexpr int kBitmapWords = 128; // selection bitmap: nb <= 4096
+constexpr int kWarpScratchWords = kBins + kBitmapWords + 2 * kMaxCand + 4;
+
+// Exact top-`budget` of a shared-memory row (one warp), lowest index on ties:
+//  1. row min and max;
+//  2. histogram over kBins bins linear in the value (a monotone map, equal
+//     values share a bin); lanes walk the row with a stride of ceil(nb/32) so
+//     that neighbouring lanes touch distant (differently valued) blocks;
+//  3. the bin b* holding the budget-th largest value and the count above it;
+//  4. everything above b* goes into a bitmap; the values of b* are gathered
+//     and ranked exactly by (order key desc, index asc) to fill the rest;
+//  5. the bitmap is written out in ascending block order.
+// A threshold bin with more than kMaxCand values falls back to the radix
+// select (same result, slower).
+__device__ __forceinline__ void warp_topk_row_binned(const float* row, int nb, int budget,
+                                                     uint32_t* scratch, int32_t* out, int lane) {
+  uint32_t* hist = scratch;                          // [kBins]
+  uint32_t* bits = hist + kBins;                     // [kBitmapWords]
+  uint32_t* cand_key = bits + kBitmapWords;          // [kMaxCand]
+  uint32_t* cand_j = cand_key + kMaxCand;            // [kMaxCand]
+  uint32_t* cand_n = cand_j + kMaxCand;              // [1]
+  float lo = INFINITY, hi = -INFINITY;
+  for (int j = lane; j < nb; j += 32) {
+    const float v = row[j];
+    lo = fminf(lo, v);
+    hi = fmaxf(hi, v);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  const float scale = (float)kBins / (hi - lo);
+  for (int b = lane; b < kBins; b += 32) hist[b] = 0u;
+  for (int w = lane; w < kBitmapWords; w += 32) bits[w] = 0u;
+  if (lane == 0) *cand_n = 0u;
+  __syncwarp();
+  const int stride = (nb + 31) >> 5;
+  auto bin_of = [&](float v) -> int {
+    const float t = (v - lo) * scale;           // monotone in v; NaN -> bin 0
+    int b = (t >= 0.f) ? (int)fminf(t, (float)(kBins - 1)) : 0;
+    return b;
+  };
+  for (int it = 0; it < stride; ++it) {
+    const int j = lane * stride + it;
+    if (j < nb) atomicAdd(&hist[bin_of(row[j])], 1u);
+  }
+  __syncwarp();
+  // Lane l owns bins kBins-1-16l .. kBins-16-16l (descending).
+  constexpr int kPer = kBins / 32;
+  int cnt[kPer];
+  int tot = 0;
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    cnt[u] = (int)hist[kBins - 1 - kPer * lane - u];
+    tot += cnt[u];
+  }
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int excl = incl - tot;
+  const unsigned ball = __ballot_sync(0xffffffffu, excl < budget && budget <= incl);
+  const int src = ball ? __ffs(ball) - 1 : 0;
+  int bstar = 0, above = 0;
+  if (lane == src) {
+    int acc = excl;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      if (acc + cnt[u] >= budget) {
+        bstar = kBins - 1 - kPer * lane - u;
+        above = acc;
+        break;
+      }
+      acc += cnt[u];
+    }
+  }
+  bstar = __shfl_sync(0xffffffffu, bstar, src);
+  above = __shfl_sync(0xffffffffu, above, src);
+  const int need = budget - above;
+  const int in_bin = (int)hist[bstar];
+  if (in_bin > kMaxCand) {                     // crowded threshold bin: exact radix select
+    __syncwarp();
+    warp_topk_row(row, nb, budget, hist, out, lane);
+    return;
+  }
+  for (int it = 0; it < stride; ++it) {
+    const int j = lane * stride + it;
+    if (j < nb) {
+      const float v = row[j];
+      const int b = bin_of(v);
+      if (b > bstar) {
+        atomicOr(&bits[j >> 5], 1u << (j & 31));
+      } else if (b == bstar) {
+        const uint32_t slot = atomicAdd(cand_n, 1u);
+        cand_key[slot] = order_key(v);
+        cand_j[slot] = (uint32_t)j;
+      }
+    }
+  }
+  __syncwarp();
+  // Rank the candidates: larger key first, lower index first on equal keys.
+  for (int c = lane; c < in_bin; c += 32) {
+    const uint32_t kc = cand_key[c], jc = cand_j[c];
+    int rank = 0;
+    for (int o = 0; o < in_bin; ++o) {
+      const uint32_t ko = cand_key[o], jo = cand_j[o];
+      rank += (ko > kc || (ko == kc && jo < jc)) ? 1 : 0;
+    }
+    if (rank < need) atomicOr(&bits[jc >> 5], 1u << (jc & 31));
+  }
+  __syncwarp();
+  // Bitmap -> ascending list.
+  const int words = (nb + 31) >> 5;
+  int base = 0;
+  for (int w0 = 0; w0 < words; w0 += 32) {
+    const int w = w0 + lane;
+    uint32_t m = (w < words) ? bits[w] : 0u;
+    const int c = __popc(m);
+    int inc = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    int pos = base + inc - c;
+    while (m) {
+      const int bit = __ffs(m) - 1;
+      m &= m - 1u;
+      out[pos++] = w * 32 + bit;
+    }
+    base += __shfl_sync(0xffffffffu, inc, 31);
+  }
+}
+
 // CTA = one head and R consecutive query blocks; 256 threads.  Scores of the
 // R rows over all nb key blocks stay in shared memory.
 template <int R>
@@ -219,8 +360,8 @@ __global__ void __launch_bounds__(256, 1) score_topk_kernel(const ScoreArgs a) {
   extern __shared__ __align__(16) float sm[];
   float* kt = sm;                          // [64][TK]
   float* qs = kt + kHeadDim * TK;          // [64][R]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(qs + kHeadDim * R);  // [8][256]
-  float* scores = reinterpret_cast<float*>(hist + 8 * 256);          // [R][nb_pad]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(qs + kHeadDim * R);  // [8][kWarpScratchWords]
+  float* scores = reinterpret_cast<float*>(hist + 8 * kWarpScratchWords);  // [R][nb_pad]
 
   const int h = blockIdx.x / a.tiles_per_head;
   const int i0 = (blockIdx.x % a.tiles_per_head) * R;
@@ -271,7 +412,7 @@ __global__ void __launch_bounds__(256, 1) score_topk_kernel(const ScoreArgs a) {
   __syncthreads();
 
   // One warp per row.
-  uint32_t* whist = hist + warp * 256;
+  uint32_t* whist = hist + warp * kWarpScratchWords;
 #pragma unroll 1
   for (int r = warp; r < R; r += 8) {
     const int i = i0 + r;
@@ -290,14 +431,14 @@ __global__ void __launch_bounds__(256, 1) score_topk_kernel(const ScoreArgs a) {
       for (int j = lane; j < nb; j += 32) row[j] = expf(row[j] - m) / z + a.lambda * ch[j];
       __syncwarp();
     }
-    warp_topk_row(row, nb, a.budget, whist, a.idx + ((size_t)h * nb + i) * a.budget, lane);
+    warp_topk_row_binned(row, nb, a.budget, whist, a.idx + ((size_t)h * nb + i) * a.budget, lane);
   }
 }
 
 template <int R>
 size_t score_smem_bytes(int nb_pad) {
-  return sizeof(float) * ((size_t)kHeadDim * (2048 / R) + (size_t)kHeadDim * R + 8 * 256 +
-                          (size_t)R * nb_pad);
+  return sizeof(float) * ((size_t)kHeadDim * (2048 / R) + (size_t)kHeadDim * R +
+                          8 * (size_t)kWarpScratchWords + (size_t)R * nb_pad);
 }
 
 template <int R>
