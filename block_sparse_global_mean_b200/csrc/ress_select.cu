@@ -135,11 +135,14 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 }
 
 struct ScoreArgs {
+  DeviceError* err;
   const float* qbar;     // [H][nb][64]
   const float* kbar_t;   // [H][64][nb_pad]
   const float* contrast; // [H][nb] or null
   int32_t* idx;          // [H][nb][budget]
   int heads, nb, nb_pad, budget, tiles_per_head;
+  int row_stride;         // floats between score rows in shared memory
+  int stages;             // ring stages
   float lambda;
 };
 
@@ -212,55 +215,98 @@ __device__ __forceinline__ void warp_topk_row(const float* row, int nb, int budg
   }
 }
 
-constexpr int kBins = 512;        // linear histogram bins over [row min, row max]
-constexpr int kMaxCand = 64;      // candidates resolved exactly in the threshold bin
-constexpr int kBitmapWords = 128; // selection bitmap: nb <= 4096
-constexpr int kWarpScratchWords = kBins + kBitmapWords + 2 * kMaxCand + 4;
+constexpr int kBins = 512;        // histogram bins, linear in the value over [row min, row max]
+constexpr int kMaxCand = 64;      // values of the threshold bin that are ranked exactly
+constexpr int kBitmapWords = 128; // kept-block bitmap: nb <= 4096
+constexpr int kWarpScratchWords = kBins + kBitmapWords + 2 * kMaxCand;
 
-// Exact top-`budget` of a shared-memory row (one warp), lowest index on ties:
-//  1. row min and max;
-//  2. histogram over kBins bins linear in the value (a monotone map, equal
-//     values share a bin); lanes walk the row with a stride of ceil(nb/32) so
-//     that neighbouring lanes touch distant (differently valued) blocks;
-//  3. the bin b* holding the budget-th largest value and the count above it;
-//  4. everything above b* goes into a bitmap; the values of b* are gathered
-//     and ranked exactly by (order key desc, index asc) to fill the rest;
-//  5. the bitmap is written out in ascending block order.
+// Shared-memory histogram increment; the result is not returned.
+__device__ __forceinline__ void red_add_shared(uint32_t addr, uint32_t v) {
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(addr), "r"(v));
+}
+
+// Bin of v: round((v - lo) * scale) clamped to [0, kBins - 1], through the
+// round-to-nearest of adding 1.5 * 2^23.  Monotone non-decreasing in v (NaN
+// -> 0, below every number, as in order_key); always a valid index.
+__device__ __forceinline__ uint32_t value_bin(float v, float lo, float scale) {
+  const float d = fmaxf(v - lo, 0.f);
+  const uint32_t b = __float_as_uint(fmaf(d, scale, 12582912.0f)) - 0x4B400000u;
+  return min(b, (uint32_t)(kBins - 1));
+}
+
+// Exact top-`budget` of a shared-memory row (one warp), lowest index on ties.
+//  1. row min and max, and
+//  2. a histogram over kBins bins linear in the value, both with lane l
+//     reading the contiguous run [l * run, (l + 1) * run) as float4 (run =
+//     4 x an odd number: the eight lanes of one 128-bit access phase hit
+//     disjoint banks, and neighbouring lanes hold distant, differently valued
+//     blocks, so their histogram increments rarely collide); the bin b*
+//     holding the budget-th largest value and the count above it follow from
+//     a scan over the bins;
+//  3. the values of b* are gathered in ascending index order (32 consecutive
+//     blocks per lane step, ballot compaction) and ranked exactly by (order
+//     key desc, index asc);
+//  4. a last pass over 32 consecutive blocks per step writes every block
+//     above b* and the winners of b*, compacted by ballot, in ascending order.
+// Every pass issues four independent loads before using any of them, so that
+// one warp keeps several shared-memory accesses in flight.
 // A threshold bin with more than kMaxCand values falls back to the radix
 // select (same result, slower).
 __device__ __forceinline__ void warp_topk_row_binned(const float* row, int nb, int budget,
                                                      uint32_t* scratch, int32_t* out, int lane) {
   uint32_t* hist = scratch;                          // [kBins]
-  uint32_t* bits = hist + kBins;                     // [kBitmapWords]
-  uint32_t* cand_key = bits + kBitmapWords;          // [kMaxCand]
+  uint32_t* wins = hist + kBins;                     // [kBitmapWords] kept-block bitmap
+  uint32_t* cand_key = wins + kBitmapWords;          // [kMaxCand]
   uint32_t* cand_j = cand_key + kMaxCand;            // [kMaxCand]
-  uint32_t* cand_n = cand_j + kMaxCand;              // [1]
+  const uint32_t hist_s = smem_addr(hist);
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int run = 4 * ((((nb + 31) >> 5) + 3) >> 2 | 1);
+  const int j0 = min(lane * run, nb);
+  const int j1 = min(j0 + run, nb);
+  const int n4 = (j1 - j0) >> 2;          // float4s of the run; [j0 + 4 n4, j1) one by one
+  const float4* run4 = reinterpret_cast<const float4*>(row + j0);
   float lo = INFINITY, hi = -INFINITY;
-  for (int j = lane; j < nb; j += 32) {
-    const float v = row[j];
-    lo = fminf(lo, v);
-    hi = fmaxf(hi, v);
+  for (int g = 0; g < n4; g += 4) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = run4[min(g + u, n4 - 1)];   // repeats are harmless
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      lo = fminf(lo, fminf(fminf(v[u].x, v[u].y), fminf(v[u].z, v[u].w)));
+      hi = fmax3(hi, fmaxf(v[u].x, v[u].y), fmaxf(v[u].z, v[u].w));
+    }
+  }
+  for (int j = j0 + 4 * n4; j < j1; ++j) {
+    lo = fminf(lo, row[j]);
+    hi = fmaxf(hi, row[j]);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
     hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
   }
-  const float scale = (float)kBins / (hi - lo);
-  for (int b = lane; b < kBins; b += 32) hist[b] = 0u;
-  for (int w = lane; w < kBitmapWords; w += 32) bits[w] = 0u;
-  if (lane == 0) *cand_n = 0u;
+  float scale = (float)(kBins - 1) / (hi - lo);
+  if (!(scale < INFINITY)) scale = 0.f;   // constant row (or non-finite range): one bin
+  for (int b = 4 * lane; b < kBins; b += 128)
+    *reinterpret_cast<uint4*>(hist + b) = make_uint4(0u, 0u, 0u, 0u);
+  for (int w = 4 * lane; w < kBitmapWords; w += 128)
+    *reinterpret_cast<uint4*>(wins + w) = make_uint4(0u, 0u, 0u, 0u);
   __syncwarp();
-  const int stride = (nb + 31) >> 5;
-  auto bin_of = [&](float v) -> int {
-    const float t = (v - lo) * scale;           // monotone in v; NaN -> bin 0
-    int b = (t >= 0.f) ? (int)fminf(t, (float)(kBins - 1)) : 0;
-    return b;
-  };
-  for (int it = 0; it < stride; ++it) {
-    const int j = lane * stride + it;
-    if (j < nb) atomicAdd(&hist[bin_of(row[j])], 1u);
+  for (int g = 0; g < n4; g += 4) {
+    float4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = run4[min(g + u, n4 - 1)];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (g + u < n4) {
+        red_add_shared(hist_s + 4u * value_bin(v[u].x, lo, scale), 1u);
+        red_add_shared(hist_s + 4u * value_bin(v[u].y, lo, scale), 1u);
+        red_add_shared(hist_s + 4u * value_bin(v[u].z, lo, scale), 1u);
+        red_add_shared(hist_s + 4u * value_bin(v[u].w, lo, scale), 1u);
+      }
+    }
   }
+  for (int j = j0 + 4 * n4; j < j1; ++j) red_add_shared(hist_s + 4u * value_bin(row[j], lo, scale), 1u);
   __syncwarp();
   // Lane l owns bins kBins-1-16l .. kBins-16-16l (descending).
   constexpr int kPer = kBins / 32;
@@ -280,20 +326,20 @@ __device__ __forceinline__ void warp_topk_row_binned(const float* row, int nb, i
   const int excl = incl - tot;
   const unsigned ball = __ballot_sync(0xffffffffu, excl < budget && budget <= incl);
   const int src = ball ? __ffs(ball) - 1 : 0;
-  int bstar = 0, above = 0;
+  int bstar_i = 0, above = 0;
   if (lane == src) {
     int acc = excl;
 #pragma unroll
     for (int u = 0; u < kPer; ++u) {
       if (acc + cnt[u] >= budget) {
-        bstar = kBins - 1 - kPer * lane - u;
+        bstar_i = kBins - 1 - kPer * lane - u;
         above = acc;
         break;
       }
       acc += cnt[u];
     }
   }
-  bstar = __shfl_sync(0xffffffffu, bstar, src);
+  const uint32_t bstar = (uint32_t)__shfl_sync(0xffffffffu, bstar_i, src);
   above = __shfl_sync(0xffffffffu, above, src);
   const int need = budget - above;
   const int in_bin = (int)hist[bstar];
@@ -302,22 +348,39 @@ __device__ __forceinline__ void warp_topk_row_binned(const float* row, int nb, i
     warp_topk_row(row, nb, budget, hist, out, lane);
     return;
   }
-  for (int it = 0; it < stride; ++it) {
-    const int j = lane * stride + it;
-    if (j < nb) {
-      const float v = row[j];
-      const int b = bin_of(v);
-      if (b > bstar) {
-        atomicOr(&bits[j >> 5], 1u << (j & 31));
-      } else if (b == bstar) {
-        const uint32_t slot = atomicAdd(cand_n, 1u);
-        cand_key[slot] = order_key(v);
-        cand_j[slot] = (uint32_t)j;
+  // One pass, 4 x 32 consecutive blocks a step: the blocks above b* go into
+  // the bitmap (one ballot word per 32 blocks); the values of b* are gathered
+  // in ascending index order.
+  int ncand = 0;
+  for (int c0 = 0; c0 < nb; c0 += 128) {
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = row[min(c0 + 32 * u + lane, nb - 1)];
+    unsigned ma[4], mc[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t b = value_bin(v[u], lo, scale);
+      const bool valid = c0 + 32 * u + lane < nb;
+      ma[u] = __ballot_sync(0xffffffffu, valid && b > bstar);
+      mc[u] = __ballot_sync(0xffffffffu, valid && b == bstar);
+    }
+    if (lane < 4 && c0 + 32 * lane < nb)
+      wins[(c0 >> 5) + lane] = lane == 0 ? ma[0] : lane == 1 ? ma[1] : lane == 2 ? ma[2] : ma[3];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (mc[u] != 0u) {                       // warp-uniform; rare
+        if ((mc[u] >> lane) & 1u) {
+          const int slot = ncand + __popc(mc[u] & lt_mask);
+          cand_key[slot] = order_key(v[u]);
+          cand_j[slot] = (uint32_t)(c0 + 32 * u + lane);
+        }
+        ncand += __popc(mc[u]);
       }
     }
   }
   __syncwarp();
-  // Rank the candidates: larger key first, lower index first on equal keys.
+  // Rank the candidates: larger key first, lower index first on equal keys;
+  // the winners join the bitmap.
   for (int c = lane; c < in_bin; c += 32) {
     const uint32_t kc = cand_key[c], jc = cand_j[c];
     int rank = 0;
@@ -325,131 +388,233 @@ __device__ __forceinline__ void warp_topk_row_binned(const float* row, int nb, i
       const uint32_t ko = cand_key[o], jo = cand_j[o];
       rank += (ko > kc || (ko == kc && jo < jc)) ? 1 : 0;
     }
-    if (rank < need) atomicOr(&bits[jc >> 5], 1u << (jc & 31));
+    if (rank < need) atomicOr(&wins[jc >> 5], 1u << (jc & 31));
   }
   __syncwarp();
-  // Bitmap -> ascending list.
+  // Emit the bitmap in ascending order, four words a step.
   const int words = (nb + 31) >> 5;
   int base = 0;
-  for (int w0 = 0; w0 < words; w0 += 32) {
-    const int w = w0 + lane;
-    uint32_t m = (w < words) ? bits[w] : 0u;
-    const int c = __popc(m);
-    int inc = c;
+  for (int w0 = 0; w0 < words; w0 += 4) {
+    const uint4 m4 = *reinterpret_cast<const uint4*>(wins + w0);   // words >= `words` are 0
+    const uint32_t m[4] = {m4.x, m4.y, m4.z, m4.w};
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, inc, o);
-      if (lane >= o) inc += y;
+    for (int u = 0; u < 4; ++u) {
+      if ((m[u] >> lane) & 1u) out[base + __popc(m[u] & lt_mask)] = 32 * (w0 + u) + lane;
+      base += __popc(m[u]);
     }
-    int pos = base + inc - c;
-    while (m) {
-      const int bit = __ffs(m) - 1;
-      m &= m - 1u;
-      out[pos++] = w * 32 + bit;
-    }
-    base += __shfl_sync(0xffffffffu, inc, 31);
   }
 }
 
-// CTA = one head and R consecutive query blocks; 256 threads.  Scores of the
-// R rows over all nb key blocks stay in shared memory.
+// CTA = one head and R consecutive query blocks: R consumer warps and one
+// producer warp.  The pooled keys stream through a ring of 16 KB shared-memory
+// stages, each [4 d][1024 keys] fp32, filled by bulk copies that the producer
+// issues as soon as every consumer warp has released the stage.  Consumer
+// warp w handles rows 8 (w / 8) .. 8 (w / 8) + 7; its lane l accumulates them
+// against keys 128 (w % 8) + 4 l .. + 3 of the tile, two rows per packed fp32
+// FMA, d in ascending order.  The R score rows (all nb key blocks) stay in
+// shared memory.  Then each consumer warp selects the top `budget` of one row.
+constexpr uint32_t kStageBytes = 16384;
+constexpr int kScoreTK = 1024;                          // keys per tile
+constexpr int kScoreTD = kStageBytes / (4 * kScoreTK);  // d per stage (4)
+constexpr int kStagesPerTile = kHeadDim / kScoreTD;
+
 template <int R>
-__global__ void __launch_bounds__(256, 1) score_topk_kernel(const ScoreArgs a) {
-  constexpr int TK = 2048 / R;   // key blocks per shared-memory tile
-  constexpr int KP = TK / 2;     // key pairs per row group
+struct ScoreCfg {
+  static constexpr int kConsumers = 32 * R;              // one warp per row
+  static constexpr int kThreads = kConsumers + 32;       // + producer warp
+  static_assert(R % 8 == 0 && (R / 8) * 8 * 128 == kScoreTK * (R / 8), "eight warps per row group");
+  // The top-k scratch of the R consumer warps reuses the stage ring, which
+  // has at least 4 stages for R = 16 and 2 for R = 8.
+  static_assert(R * kWarpScratchWords * 4 <= (R == 16 ? 4 : 2) * (int)kStageBytes,
+                "top-k scratch fits the stage ring");
+};
+
+// Registers are capped so that five warps of one SM sub-partition fit its
+// register file (5 x 32 x 96 <= 16,384) at 544 threads.
+template <int R>
+__global__ void __maxnreg__(96) score_topk_kernel(const ScoreArgs a) {
+  using C = ScoreCfg<R>;
+  constexpr int TK = kScoreTK, TD = kScoreTD;
   extern __shared__ __align__(16) float sm[];
-  float* kt = sm;                          // [64][TK]
-  float* qs = kt + kHeadDim * TK;          // [64][R]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(qs + kHeadDim * R);  // [8][kWarpScratchWords]
-  float* scores = reinterpret_cast<float*>(hist + 8 * kWarpScratchWords);  // [R][nb_pad]
+  const int S = a.stages;
+  float* stages = sm;                                    // [S][TD][TK]; top-k scratch later
+  float* qs = stages + (size_t)S * TD * TK;              // [64][R]
+  float* scores = qs + kHeadDim * R;                     // [R][row_stride]
+  const int nb = a.nb, nb_pad = a.nb_pad, rs = a.row_stride;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(scores + (size_t)R * rs);   // full[S], empty[S]
+  int* abortf = reinterpret_cast<int*>(bars + 2 * S);
 
   const int h = blockIdx.x / a.tiles_per_head;
   const int i0 = (blockIdx.x % a.tiles_per_head) * R;
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const int nb = a.nb, nb_pad = a.nb_pad;
+  const int n_tiles = (nb_pad + TK - 1) / TK;
+  const int n_seq = n_tiles * kStagesPerTile;
+  const float* kbt = a.kbar_t + (size_t)h * kHeadDim * nb_pad;
+  const uint32_t full0 = smem_addr(&bars[0]);
+  const uint32_t empty0 = smem_addr(&bars[S]);
 
-  for (int e = tid; e < R * kHeadDim; e += 256) {
+  if (tid == 0) {
+    for (int st = 0; st < S; ++st) {
+      mbar_init(full0 + 8u * st, 1);
+      mbar_init(empty0 + 8u * st, R);
+    }
+    *abortf = 0;
+    fence_mbarrier_init();
+  }
+  for (int e = tid; e < R * kHeadDim; e += C::kThreads) {
     const int r = e / kHeadDim, d = e % kHeadDim;
     qs[d * R + r] = (i0 + r < nb) ? a.qbar[((size_t)h * nb + i0 + r) * kHeadDim + d] : 0.f;
   }
-  const int rg = tid / KP;   // rows 4*rg .. 4*rg+3
-  const int kp = tid % KP;   // key blocks 2*kp, 2*kp+1 of the tile
-  const float* kbt = a.kbar_t + (size_t)h * kHeadDim * nb_pad;
+  __syncthreads();
+
+  if (warp == R) {
+    // Producer: stage seq holds d rows TD*(seq % kStagesPerTile) .. +TD-1 of
+    // tile seq / kStagesPerTile (its keys below nb_pad).
+    int issued = 0;
+    for (int seq = 0; seq < n_seq; ++seq) {
+      const int st = seq % S;
+      const uint32_t k = (uint32_t)(seq / S);
+      bool ok = true;
+      if (seq >= S) ok = mbar_wait(empty0 + 8u * st, (k - 1u) & 1u, abortf, a.err, 72);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const int t = seq / kStagesPerTile, dq = seq % kStagesPerTile;
+      const int keys = min(TK, nb_pad - t * TK);        // a multiple of 256
+      const uint32_t full = full0 + 8u * st;
+      if (lane == 0) mbar_arrive_expect_tx(full, (uint32_t)(TD * keys * 4));
+      __syncwarp();
+      if (lane < TD)
+        bulk_load(smem_addr(stages + ((size_t)st * TD + lane) * TK),
+                  kbt + (size_t)(TD * dq + lane) * nb_pad + (size_t)t * TK, (uint32_t)keys * 4u,
+                  full);
+      issued = seq + 1;
+    }
+    // Copies still in flight (only after a timeout) land before the buffers
+    // are reused or released.
+    if (lane == 0)
+      for (int seq = issued > S ? issued - S : 0; seq < issued; ++seq)
+        mbar_wait_drain(full0 + 8u * (seq % S), (uint32_t)(seq / S) & 1u, a.err, 73);
+  } else {
+    const int rg = warp >> 3;                       // rows 8 rg .. 8 rg + 7
+    const int kw = 128 * (warp & 7) + 4 * lane;     // first of this lane's four keys in a tile
+    bool ok = true;
 #pragma unroll 1
-  for (int j0 = 0; j0 < nb; j0 += TK) {
-    __syncthreads();
-    for (int e = tid; e < kHeadDim * (TK / 4); e += 256) {
-      const int d = e / (TK / 4), c4 = e % (TK / 4);
-      reinterpret_cast<float4*>(kt + d * TK)[c4] =
-          reinterpret_cast<const float4*>(kbt + (size_t)d * nb_pad + j0)[c4];
-    }
-    __syncthreads();
-    float acc[4][2];
+    for (int t = 0; t < n_tiles && ok; ++t) {
+      // Warps whose 128 keys all lie beyond nb only keep the stage protocol.
+      const bool active = t * TK + 128 * (warp & 7) < nb;
+      float2 acc[4][4];   // acc[p][u] = rows (8 rg + 2p, 8 rg + 2p + 1) x key u
 #pragma unroll
-    for (int r = 0; r < 4; ++r) acc[r][0] = acc[r][1] = 0.f;
-#pragma unroll 16
-    for (int d = 0; d < kHeadDim; ++d) {
-      const float4 qv = *reinterpret_cast<const float4*>(qs + d * R + 4 * rg);
-      const float2 kv = *reinterpret_cast<const float2*>(kt + d * TK + 2 * kp);
-      acc[0][0] = fmaf(qv.x, kv.x, acc[0][0]);
-      acc[0][1] = fmaf(qv.x, kv.y, acc[0][1]);
-      acc[1][0] = fmaf(qv.y, kv.x, acc[1][0]);
-      acc[1][1] = fmaf(qv.y, kv.y, acc[1][1]);
-      acc[2][0] = fmaf(qv.z, kv.x, acc[2][0]);
-      acc[2][1] = fmaf(qv.z, kv.y, acc[2][1]);
-      acc[3][0] = fmaf(qv.w, kv.x, acc[3][0]);
-      acc[3][1] = fmaf(qv.w, kv.y, acc[3][1]);
-    }
-    const int j = j0 + 2 * kp;
+      for (int p = 0; p < 4; ++p)
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      float* srow = scores + (size_t)(4 * rg + r) * nb_pad;
-      if (j < nb) srow[j] = acc[r][0] * 0.125f;       // 1 / sqrt(64), exact
-      if (j + 1 < nb) srow[j + 1] = acc[r][1] * 0.125f;
+        for (int u = 0; u < 4; ++u) acc[p][u] = make_float2(0.f, 0.f);
+#pragma unroll 1
+      for (int dq = 0; dq < kStagesPerTile; ++dq) {
+        const int seq = t * kStagesPerTile + dq;
+        const int st = seq % S;
+        ok = mbar_wait(full0 + 8u * st, (uint32_t)(seq / S) & 1u, abortf, a.err, 70);
+        if (!__all_sync(0xffffffffu, ok)) {
+          ok = false;
+          break;
+        }
+        if (active) {
+          const float* kb = stages + (size_t)st * TD * TK + kw;
+          const float* qb = qs + TD * dq * R + 8 * rg;
+#pragma unroll
+          for (int dd = 0; dd < TD; ++dd) {
+            const float4 kv = *reinterpret_cast<const float4*>(kb + dd * TK);
+            const float4 q0 = *reinterpret_cast<const float4*>(qb + dd * R);
+            const float4 q1 = *reinterpret_cast<const float4*>(qb + dd * R + 4);
+            const float2 qp[4] = {make_float2(q0.x, q0.y), make_float2(q0.z, q0.w),
+                                  make_float2(q1.x, q1.y), make_float2(q1.z, q1.w)};
+            const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const float2 ku = make_float2(kk[u], kk[u]);
+#pragma unroll
+              for (int p = 0; p < 4; ++p) acc[p][u] = ffma2(qp[p], ku, acc[p][u]);
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8u * st);
+      }
+      if (!ok || !active) continue;
+      const int j = t * TK + kw;
+      // 1 / sqrt(64) = 0.125 is exact.
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        float* r0 = scores + (size_t)(8 * rg + 2 * p) * rs;
+        float* r1 = r0 + rs;
+        if (j + 3 < nb) {
+          *reinterpret_cast<float4*>(r0 + j) = make_float4(acc[p][0].x * 0.125f, acc[p][1].x * 0.125f,
+                                                           acc[p][2].x * 0.125f, acc[p][3].x * 0.125f);
+          *reinterpret_cast<float4*>(r1 + j) = make_float4(acc[p][0].y * 0.125f, acc[p][1].y * 0.125f,
+                                                           acc[p][2].y * 0.125f, acc[p][3].y * 0.125f);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (j + u < nb) {
+              r0[j + u] = acc[p][u].x * 0.125f;
+              r1[j + u] = acc[p][u].y * 0.125f;
+            }
+          }
+        }
+      }
     }
   }
   __syncthreads();
-
-  // One warp per row.
-  uint32_t* whist = hist + warp * kWarpScratchWords;
-#pragma unroll 1
-  for (int r = warp; r < R; r += 8) {
-    const int i = i0 + r;
-    if (i >= nb) break;
-    float* row = scores + (size_t)r * nb_pad;
-    if (a.lambda != 0.f) {
-      float m = -INFINITY;
-      for (int j = lane; j < nb; j += 32) m = fmaxf(m, row[j]);
+  if (*abortf != 0 || warp >= R) return;
+  // One warp per row; the stage buffers now hold each warp's top-k scratch.
+  const int i = i0 + warp;
+  if (i >= nb) return;
+  uint32_t* whist = reinterpret_cast<uint32_t*>(stages) + warp * kWarpScratchWords;
+  float* row = scores + (size_t)warp * rs;
+  if (a.lambda != 0.f) {
+    float m = -INFINITY;
+    for (int j = lane; j < nb; j += 32) m = fmaxf(m, row[j]);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      float z = 0.f;
-      for (int j = lane; j < nb; j += 32) z += expf(row[j] - m);
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float z = 0.f;
+    for (int j = lane; j < nb; j += 32) z += expf(row[j] - m);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-      const float* ch = a.contrast + (size_t)h * nb;
-      for (int j = lane; j < nb; j += 32) row[j] = expf(row[j] - m) / z + a.lambda * ch[j];
-      __syncwarp();
-    }
-    warp_topk_row_binned(row, nb, a.budget, whist, a.idx + ((size_t)h * nb + i) * a.budget, lane);
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    const float* ch = a.contrast + (size_t)h * nb;
+    for (int j = lane; j < nb; j += 32) row[j] = expf(row[j] - m) / z + a.lambda * ch[j];
+    __syncwarp();
   }
+  warp_topk_row_binned(row, nb, a.budget, whist, a.idx + ((size_t)h * nb + i) * a.budget, lane);
+}
+
+// Shared memory of score_topk_kernel<R> with `stages` ring stages and score
+// rows of `row_stride` floats.
+template <int R>
+size_t score_smem_bytes(int stages, int row_stride) {
+  return (size_t)stages * kStageBytes +
+         sizeof(float) * ((size_t)kHeadDim * R + (size_t)R * row_stride) +
+         2 * sizeof(uint64_t) * (size_t)stages + 16;
+}
+
+constexpr size_t kMaxSmem = 227 * 1024;
+constexpr int kMaxStages = 6;
+
+// Deepest ring (up to kMaxStages) that fits; 0 if fewer than `min_stages` fit.
+template <int R>
+int score_stages(int row_stride, int min_stages) {
+  for (int s = kMaxStages; s >= min_stages; --s)
+    if (score_smem_bytes<R>(s, row_stride) <= kMaxSmem) return s;
+  return 0;
 }
 
 template <int R>
-size_t score_smem_bytes(int nb_pad) {
-  return sizeof(float) * ((size_t)kHeadDim * (2048 / R) + (size_t)kHeadDim * R +
-                          8 * (size_t)kWarpScratchWords + (size_t)R * nb_pad);
-}
-
-template <int R>
-ress_status launch_score(const ScoreArgs& a0, cudaStream_t st) {
+ress_status launch_score(const ScoreArgs& a0, int stages, cudaStream_t st) {
   ScoreArgs a = a0;
   a.tiles_per_head = (a.nb + R - 1) / R;
-  const size_t smem = score_smem_bytes<R>(a.nb_pad);
-  if (ress_status st_ = record_cuda(cudaFuncSetAttribute(score_topk_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem)))
+  a.stages = stages;
+  const size_t smem = score_smem_bytes<R>(stages, a.row_stride);
+  if (ress_status st_ = record_cuda(cudaFuncSetAttribute(
+          score_topk_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
     return st_;
-  score_topk_kernel<R><<<a.heads * a.tiles_per_head, 256, smem, st>>>(a);
+  score_topk_kernel<R><<<a.heads * a.tiles_per_head, ScoreCfg<R>::kThreads, smem, st>>>(a);
   return record_cuda(cudaGetLastError());
 }
 
@@ -509,6 +674,8 @@ ress_status launch_select(const Geometry& g, const void* q, const void* k, const
     if (ress_status st_ = record_cuda(cudaGetLastError())) return st_;
   }
   ScoreArgs sa{};
+  sa.err = device_error_ptr();
+  if (sa.err == nullptr) return RESS_ERR_CUDA;
   sa.qbar = qbar;
   sa.kbar_t = kbar_t;
   sa.contrast = contrast;
@@ -518,8 +685,15 @@ ress_status launch_select(const Geometry& g, const void* q, const void* k, const
   sa.nb_pad = g.nb_pad;
   sa.budget = budget;
   sa.lambda = lambda;
-  if (g.nb <= 2304) return launch_score<16>(sa, st);
-  return launch_score<8>(sa, st);
+  sa.row_stride = (g.nb + 3) & ~3;
+  // Sixteen rows per CTA while at least four stages fit next to the score rows
+  // (nb <= 2,304), else eight.  The stage ring also holds the top-k scratch of
+  // every consumer warp afterwards.
+  const int s16 = score_stages<16>(sa.row_stride, 4);
+  if (s16 != 0) return launch_score<16>(sa, s16, st);
+  const int s8 = score_stages<8>(sa.row_stride, 2);
+  if (s8 == 0) return RESS_ERR_UNSUPPORTED;
+  return launch_score<8>(sa, s8, st);
 }
 
 }  // namespace ress

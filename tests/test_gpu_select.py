@@ -87,3 +87,39 @@ def test_budget_extremes_on_odd_block_count(budget, ress_gpu):
     _check_errors(ress_gpu)
     ref, sc = oracle.select_blocks(np64(q), np64(k), None, B, budget, 0.0, return_scores=True)
     assert_mask_parity(idx.cpu().numpy(), ref, sc["logits"], budget, max_excused_frac=0.0)
+
+
+def _random_case(nb, heads, block, seed):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(nb * block, heads, 64, generator=g).to(torch.bfloat16)
+    k = torch.randn(nb * block, heads, 64, generator=g).to(torch.bfloat16)
+    return q, k
+
+
+@pytest.mark.parametrize("nb,budget", [(13, 5), (2533, 253), (4096, 409)])
+def test_row_lengths_and_both_tile_shapes(nb, budget, ress_gpu):
+    """Odd row lengths (a ragged last run per lane), the eight-row CTA used
+    above 2,532 blocks, and the largest supported grid (4,096 blocks)."""
+    q, k = _random_case(nb, 1, 64, seed=nb)
+    idx = ress_gpu.ress_select_blocks(q.cuda(), k.cuda(), None, budget, 0.0, 64)
+    _check_errors(ress_gpu)
+    ref, sc = oracle.select_blocks(np64(q), np64(k), None, 64, budget, 0.0, return_scores=True)
+    assert_mask_parity(idx.cpu().numpy(), ref, sc["logits"], budget)
+
+
+def test_crowded_threshold_bin_and_constant_rows(ress_gpu):
+    """Many bitwise-equal pooled scores around the budget-th value (the
+    threshold bin holds far more than the exactly ranked candidates), and
+    all-zero queries whose rows are constant: the lowest indices win."""
+    nb, B, budget = 300, 64, 100
+    g = torch.Generator().manual_seed(7)
+    k = torch.randn(nb * B, 2, 64, generator=g)
+    k[40 * B:] = k[:B].repeat(nb - 40, 1, 1)                 # blocks 40.. copy block 0
+    q = torch.randn(nb * B, 2, 64, generator=g)
+    q[:, 1] = 0.0                                            # head 1: every score is 0
+    q, k = q.to(torch.bfloat16), k.to(torch.bfloat16)
+    idx = ress_gpu.ress_select_blocks(q.cuda(), k.cuda(), None, budget, 0.0, B).cpu().numpy()
+    _check_errors(ress_gpu)
+    ref, sc = oracle.select_blocks(np64(q), np64(k), None, B, budget, 0.0, return_scores=True)
+    assert_mask_parity(idx, ref, sc["logits"], budget, max_excused_frac=0.0)
+    assert (idx[1] == np.arange(budget)[None, :]).all()
