@@ -405,34 +405,36 @@ __device__ __forceinline__ void warp_topk_row_binned(const float* row, int nb, i
   }
 }
 
-// CTA = one head and R consecutive query blocks: R consumer warps and one
-// producer warp.  The pooled keys stream through a ring of 16 KB shared-memory
-// stages, each [4 d][1024 keys] fp32, filled by bulk copies that the producer
-// issues as soon as every consumer warp has released the stage.  Consumer
-// warp w handles rows 8 (w / 8) .. 8 (w / 8) + 7; its lane l accumulates them
-// against keys 128 (w % 8) + 4 l .. + 3 of the tile, two rows per packed fp32
-// FMA, d in ascending order.  The R score rows (all nb key blocks) stay in
-// shared memory.  Then each consumer warp selects the top `budget` of one row.
+// CTA = one head and R consecutive query blocks.  The pooled keys stream
+// through a ring of 16 KB shared-memory stages, each [4 d][1024 keys] fp32,
+// filled by bulk copies that the producer (the last warp) issues as soon as
+// the eight score warps have released the stage.  Lane l of score warp w
+// accumulates all R rows against keys 128 w + 4 l .. + 3 of the tile, two
+// rows per packed fp32 FMA, d in ascending order; the R score rows (all nb
+// key blocks) stay in shared memory.  Then every warp 0 .. R-1 (the producer
+// included when R = 16) selects the top `budget` of one row.
 constexpr uint32_t kStageBytes = 16384;
 constexpr int kScoreTK = 1024;                          // keys per tile
 constexpr int kScoreTD = kStageBytes / (4 * kScoreTK);  // d per stage (4)
 constexpr int kStagesPerTile = kHeadDim / kScoreTD;
+constexpr int kScoreWarps = 8;                          // warps that compute scores
+static_assert(kScoreWarps * 32 * 4 == kScoreTK, "four keys per score lane");
 
 template <int R>
 struct ScoreCfg {
-  static constexpr int kConsumers = 32 * R;              // one warp per row
-  static constexpr int kThreads = kConsumers + 32;       // + producer warp
-  static_assert(R % 8 == 0 && (R / 8) * 8 * 128 == kScoreTK * (R / 8), "eight warps per row group");
-  // The top-k scratch of the R consumer warps reuses the stage ring, which
-  // has at least 4 stages for R = 16 and 2 for R = 8.
+  static constexpr int kWarps = R > kScoreWarps ? R : kScoreWarps + 1;
+  static constexpr int kThreads = 32 * kWarps;
+  static constexpr int kProducer = kWarps - 1;
+  // The top-k scratch of the R row warps reuses the stage ring, which has at
+  // least 4 stages for R = 16 and 2 for R = 8.
   static_assert(R * kWarpScratchWords * 4 <= (R == 16 ? 4 : 2) * (int)kStageBytes,
                 "top-k scratch fits the stage ring");
 };
 
-// Registers are capped so that five warps of one SM sub-partition fit its
-// register file (5 x 32 x 96 <= 16,384) at 544 threads.
+// Registers are capped at 128 so that four warps of one SM sub-partition fit
+// its register file (4 x 32 x 128 = 16,384).
 template <int R>
-__global__ void __maxnreg__(96) score_topk_kernel(const ScoreArgs a) {
+__global__ void __maxnreg__(128) score_topk_kernel(const ScoreArgs a) {
   using C = ScoreCfg<R>;
   constexpr int TK = kScoreTK, TD = kScoreTD;
   extern __shared__ __align__(16) float sm[];
@@ -457,7 +459,7 @@ __global__ void __maxnreg__(96) score_topk_kernel(const ScoreArgs a) {
   if (tid == 0) {
     for (int st = 0; st < S; ++st) {
       mbar_init(full0 + 8u * st, 1);
-      mbar_init(empty0 + 8u * st, R);
+      mbar_init(empty0 + 8u * st, kScoreWarps);
     }
     *abortf = 0;
     fence_mbarrier_init();
@@ -468,9 +470,9 @@ __global__ void __maxnreg__(96) score_topk_kernel(const ScoreArgs a) {
   }
   __syncthreads();
 
-  if (warp == R) {
-    // Producer: stage seq holds d rows TD*(seq % kStagesPerTile) .. +TD-1 of
-    // tile seq / kStagesPerTile (its keys below nb_pad).
+  if (warp == C::kProducer) {
+    // Stage seq holds d rows TD*(seq % kStagesPerTile) .. +TD-1 of tile
+    // seq / kStagesPerTile (its keys below nb_pad).
     int issued = 0;
     for (int seq = 0; seq < n_seq; ++seq) {
       const int st = seq % S;
@@ -494,17 +496,16 @@ __global__ void __maxnreg__(96) score_topk_kernel(const ScoreArgs a) {
     if (lane == 0)
       for (int seq = issued > S ? issued - S : 0; seq < issued; ++seq)
         mbar_wait_drain(full0 + 8u * (seq % S), (uint32_t)(seq / S) & 1u, a.err, 73);
-  } else {
-    const int rg = warp >> 3;                       // rows 8 rg .. 8 rg + 7
-    const int kw = 128 * (warp & 7) + 4 * lane;     // first of this lane's four keys in a tile
+  } else if (warp < kScoreWarps) {
+    const int kw = 128 * warp + 4 * lane;           // first of this lane's four keys in a tile
     bool ok = true;
 #pragma unroll 1
     for (int t = 0; t < n_tiles && ok; ++t) {
       // Warps whose 128 keys all lie beyond nb only keep the stage protocol.
-      const bool active = t * TK + 128 * (warp & 7) < nb;
-      float2 acc[4][4];   // acc[p][u] = rows (8 rg + 2p, 8 rg + 2p + 1) x key u
+      const bool active = t * TK + 128 * warp < nb;
+      float2 acc[R / 2][4];   // acc[p][u] = rows (2p, 2p + 1) x key u
 #pragma unroll
-      for (int p = 0; p < 4; ++p)
+      for (int p = 0; p < R / 2; ++p)
 #pragma unroll
         for (int u = 0; u < 4; ++u) acc[p][u] = make_float2(0.f, 0.f);
 #pragma unroll 1
@@ -518,20 +519,21 @@ __global__ void __maxnreg__(96) score_topk_kernel(const ScoreArgs a) {
         }
         if (active) {
           const float* kb = stages + (size_t)st * TD * TK + kw;
-          const float* qb = qs + TD * dq * R + 8 * rg;
-#pragma unroll
+          const float* qb = qs + TD * dq * R;
+#pragma unroll 2   // full unrolling spills at 128 registers
           for (int dd = 0; dd < TD; ++dd) {
             const float4 kv = *reinterpret_cast<const float4*>(kb + dd * TK);
-            const float4 q0 = *reinterpret_cast<const float4*>(qb + dd * R);
-            const float4 q1 = *reinterpret_cast<const float4*>(qb + dd * R + 4);
-            const float2 qp[4] = {make_float2(q0.x, q0.y), make_float2(q0.z, q0.w),
-                                  make_float2(q1.x, q1.y), make_float2(q1.z, q1.w)};
             const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const float2 ku = make_float2(kk[u], kk[u]);
+            for (int m = 0; m < R / 4; ++m) {
+              const float4 qv = *reinterpret_cast<const float4*>(qb + dd * R + 4 * m);
+              const float2 qa = make_float2(qv.x, qv.y), qc = make_float2(qv.z, qv.w);
 #pragma unroll
-              for (int p = 0; p < 4; ++p) acc[p][u] = ffma2(qp[p], ku, acc[p][u]);
+              for (int u = 0; u < 4; ++u) {
+                const float2 ku = make_float2(kk[u], kk[u]);
+                acc[2 * m][u] = ffma2(qa, ku, acc[2 * m][u]);
+                acc[2 * m + 1][u] = ffma2(qc, ku, acc[2 * m + 1][u]);
+              }
             }
           }
         }
@@ -542,8 +544,8 @@ __global__ void __maxnreg__(96) score_topk_kernel(const ScoreArgs a) {
       const int j = t * TK + kw;
       // 1 / sqrt(64) = 0.125 is exact.
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        float* r0 = scores + (size_t)(8 * rg + 2 * p) * rs;
+      for (int p = 0; p < R / 2; ++p) {
+        float* r0 = scores + (size_t)(2 * p) * rs;
         float* r1 = r0 + rs;
         if (j + 3 < nb) {
           *reinterpret_cast<float4*>(r0 + j) = make_float4(acc[p][0].x * 0.125f, acc[p][1].x * 0.125f,
