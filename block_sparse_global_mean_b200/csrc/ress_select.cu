@@ -50,7 +50,7 @@ __device__ __forceinline__ void accum_vec(float* acc, const uint4& v, const floa
 // grid (nb, tensors); block = vpr * phases threads; thread (col, phase) sums
 // the 16-byte column `col` of tokens phase, phase + phases, ... of its block.
 template <typename T>
-__global__ void __launch_bounds__(1024) pool_kernel(const PoolArgs a) {
+__global__ void __launch_bounds__(1024, 1) pool_kernel(const PoolArgs a) {
   constexpr int EPV = 16 / sizeof(T);
   extern __shared__ float red[];
   const int i = blockIdx.x;
@@ -59,8 +59,12 @@ __global__ void __launch_bounds__(1024) pool_kernel(const PoolArgs a) {
   const int phases = blockDim.x / vpr;
   const int col = threadIdx.x % vpr;
   const int ph = threadIdx.x / vpr;
-  const uint4* base =
-      reinterpret_cast<const uint4*>(a.src[t]) + (size_t)i * a.block * vpr + col;
+  // Picked by value: indexing the parameter arrays with t would copy them to
+  // local memory.
+  const void* src = t == 0 ? a.src[0] : (t == 1 ? a.src[1] : a.src[2]);
+  float* dst = t == 0 ? a.dst[0] : (t == 1 ? a.dst[1] : a.dst[2]);
+  const int layout = t == 0 ? a.layout[0] : (t == 1 ? a.layout[1] : a.layout[2]);
+  const uint4* base = reinterpret_cast<const uint4*>(src) + (size_t)i * a.block * vpr + col;
   float acc[EPV];
 #pragma unroll
   for (int u = 0; u < EPV; ++u) acc[u] = 0.f;
@@ -91,8 +95,7 @@ __global__ void __launch_bounds__(1024) pool_kernel(const PoolArgs a) {
   const int e0 = col * EPV;           // element within the token row (H * 64)
   const int hh = e0 / kHeadDim;
   const int dd = e0 % kHeadDim;
-  float* dst = a.dst[t];
-  if (a.layout[t] == 0) {
+  if (layout == 0) {
     float4* o = reinterpret_cast<float4*>(dst + ((size_t)hh * a.nb + i) * kHeadDim + dd);
 #pragma unroll
     for (int u = 0; u < EPV / 4; ++u)
