@@ -18,7 +18,11 @@
 // directions of the contributions, so the set drift is the norm of their sum.
 //
 // Warp roles as in the attention kernel (warp 0 TMA, warp 1 TMEM + MMA,
-// warps 2-5 exponentials and reductions); one CTA per SM (512 TMEM columns).
+// warps 2-5 exponentials and reductions).  Each CTA runs the chunk chain
+// S -> P -> C_j -> ||C_j|| serially; with 128-token blocks a CTA needs 256
+// TMEM columns (S, C, T) and two CTAs share an SM, so that one CTA's
+// exponentials overlap the other's MMAs and reductions.  With 64-token blocks
+// (two contributions per chunk) a CTA takes all 512 columns.
 #include "ress_common.cuh"
 #include "ress_internal.h"
 
@@ -32,11 +36,14 @@ constexpr int kThreads = 192;
 constexpr uint32_t kQBytes = 128 * 128;
 constexpr uint32_t kSubBytes = 64 * 128;
 constexpr uint32_t kStageBytes = 4 * kSubBytes;
-constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0;     // S (fp32) / P (bf16, cols 0..63)
 constexpr uint32_t kColC0 = 128;  // contribution of sub-block 0 (or the whole 128-key block)
 constexpr uint32_t kColC1 = 192;  // contribution of sub-block 1 (block 64 only)
-constexpr uint32_t kColT = 256;   // running sum of the contributions
+// TMEM columns and the running sum's column: 256 / 192 for 128-token blocks
+// (C1 unused), 512 / 256 for 64-token blocks.
+template <bool B128> constexpr uint32_t tmem_cols() { return B128 ? 256u : 512u; }
+template <bool B128> constexpr uint32_t col_t() { return B128 ? 192u : 256u; }
+constexpr size_t kOneCtaSmem = 116 * 1024;
 
 struct DriftParams {
   DeviceError* err;
@@ -124,7 +131,8 @@ __device__ __forceinline__ int dropped_rank(const uint32_t* kept, const uint32_t
   return j - (int)(prefix[j >> 5] + __popc(below));
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <bool B128>
+__global__ void __launch_bounds__(kThreads, B128 ? 2 : 1)
     block_drift_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const DriftParams p) {
@@ -180,7 +188,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbarrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(&ctl->tmem_base), kTmemCols);
+    tmem_alloc(smem_addr(&ctl->tmem_base), tmem_cols<B128>());
     tmem_relinquish();
   }
   for (int w = threadIdx.x; w < 2 * W; w += kThreads) keptA[w] = 0u;
@@ -335,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + kColT, tS + kk * 8, dv + (uint64_t)(kk * 128), idPV,
+            mma_ts(tmem + col_t<B128>(), tS + kk * 8, dv + (uint64_t)(kk * 128), idPV,
                    (c > 0 || kk > 0) ? 1u : 0u);
           mma_commit(bar_c);
           mma_commit(smem_addr(&ctl->kv_empty[s]));
@@ -369,23 +377,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool use0 = (m0 >> half) & 1u;
       const bool use1 = (m1 >> half) & 1u;
       if (use0 || use1) {
-        uint32_t r[4][32];
-        tmem_ld32(tS, r[0]);
-        tmem_ld32(tS + 32, r[1]);
-        tmem_ld32(tS + 64, r[2]);
-        tmem_ld32(tS + 96, r[3]);
-        tmem_ld_wait();
+        // Two halves of 64 columns; P (bf16, two per column) of half hf goes
+        // to columns 32 hf .. 32 hf + 31, below the S columns still unread.
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const bool use = (g < 2) ? use0 : use1;
-          uint32_t pk[16];
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t r[2][32];
+          tmem_ld32(tS + 64 * hf, r[0]);
+          tmem_ld32(tS + 64 * hf + 32, r[1]);
+          tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e]), kScaleLog2, neg_l));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e + 1]), kScaleLog2, neg_l));
-            pk[e] = use ? pack_bf16x2(p0, p1) : 0u;
+          for (int g = 0; g < 2; ++g) {
+            const bool use = hf == 0 ? use0 : use1;
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float p0 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e]), kScaleLog2, neg_l));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e + 1]), kScaleLog2, neg_l));
+              pk[e] = use ? pack_bf16x2(p0, p1) : 0u;
+            }
+            tmem_st16(tS + 32 * hf + 16 * g, pk);
           }
-          tmem_st16(tS + 16 * g, pk);
         }
       } else {
         uint32_t z[32];
@@ -478,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t tv[32];
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
-          tmem_ld32(tmem + kColT + lane_off + 32 * g, tv);
+          tmem_ld32(tmem + col_t<B128>() + lane_off + 32 * g, tv);
           tmem_ld_wait();
 #pragma unroll
           for (int u = 0; u < 32; ++u) {
@@ -512,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, tmem_cols<B128>());
   }
 }
 
@@ -540,11 +551,21 @@ ress_status launch_drift(const Geometry& g, const void* q, const void* k, const 
   p.set_drift = set_drift;
   const size_t smem = drift_smem_bytes(g.nb);
   if (smem > 227 * 1024) return RESS_ERR_UNSUPPORTED;   // block lists no longer fit
-  if (ress_status st_ = record_cuda(cudaFuncSetAttribute(block_drift_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem)))
-    return st_;
-  block_drift_kernel<<<(unsigned)(g.heads * p.tiles_per_head), kThreads, smem, st>>>(tq, tk, tv,
-                                                                                     p);
+  const unsigned grid = (unsigned)(g.heads * p.tiles_per_head);
+  if (g.block == 128) {
+    if (ress_status st_ = record_cuda(cudaFuncSetAttribute(
+            block_drift_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+      return st_;
+    block_drift_kernel<true><<<grid, kThreads, smem, st>>>(tq, tk, tv, p);
+  } else {
+    // All 512 TMEM columns per CTA: at least 116 KB of shared memory keeps a
+    // second CTA (which would only wait in its TMEM allocation) off the SM.
+    const size_t smem1 = smem > kOneCtaSmem ? smem : kOneCtaSmem;
+    if (ress_status st_ = record_cuda(cudaFuncSetAttribute(
+            block_drift_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)))
+      return st_;
+    block_drift_kernel<false><<<grid, kThreads, smem1, st>>>(tq, tk, tv, p);
+  }
   return record_cuda(cudaGetLastError());
 }
 
