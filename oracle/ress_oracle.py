@@ -156,6 +156,52 @@ def select_blocks(q, k, v, block: int, budget: int, lam: float = 0.0,
     return idx
 
 
+def cdf_counts(probs, tau: float) -> np.ndarray:
+    """Per row, how many blocks the cumulative (CDF) threshold keeps.
+
+    SparseVGGT keeps, for every query block, the key blocks of largest pooled
+    probability until their cumulative mass reaches a threshold (ReSS, Table S5:
+    with the similarity gate off, selection reduces to a cumulative threshold on
+    pooled query/key inner products; Table 2, row "+ CDF threshold").
+    Reading: blocks in descending probability, ties to the lower index; the
+    count is the smallest m >= 1 whose first m probabilities sum to at least
+    tau; every block when the rounded total never reaches tau.
+    """
+    p = _f64(probs)
+    nb = p.shape[-1]
+    order = np.argsort(-p, axis=-1, kind="stable")
+    cum = np.cumsum(np.take_along_axis(p, order, axis=-1), axis=-1)
+    reached = cum >= tau
+    first = np.argmax(reached, axis=-1) + 1
+    return np.where(reached.any(axis=-1), first, nb).astype(np.int32)
+
+
+def select_blocks_cdf(q, k, block: int, tau: float, capacity: int,
+                      return_scores: bool = False):
+    """Stage 1 with the CDF threshold instead of a fixed budget.
+
+    Returns (counts [H, nb] int32, idx [H, nb, capacity] int32).  Row (h, i)
+    keeps its top min(counts[h, i], capacity) blocks (by pooled probability,
+    ties to the lower index) in ascending order; the rest of the row repeats
+    its last kept block, so that idx is also a valid fixed-capacity kept list
+    (duplicates name the same block).
+    """
+    sc = selection_scores(q, k, None, block, 0.0)
+    counts = cdf_counts(sc["probs"], tau)
+    h_count, nb, _ = sc["probs"].shape
+    idx = np.zeros((h_count, nb, capacity), dtype=np.int32)
+    order = np.argsort(-sc["probs"], axis=-1, kind="stable")
+    for h in range(h_count):
+        for i in range(nb):
+            keep = min(int(counts[h, i]), capacity)
+            kept = np.sort(order[h, i, :keep])
+            idx[h, i, :keep] = kept
+            idx[h, i, keep:] = kept[-1]
+    if return_scores:
+        return counts, idx, sc
+    return counts, idx
+
+
 # ---------------------------------------------------------------------------
 # Stage 2: block-sparse attention
 # ---------------------------------------------------------------------------

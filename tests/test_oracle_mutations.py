@@ -36,6 +36,12 @@ MUTATIONS = {
     "set drift as the sum of magnitudes":
         ("return drift, float(np.sqrt((total * total).sum()))",
          "return drift, float(drift.sum())"),
+    "CDF threshold exceeded instead of reached":
+        ("reached = cum >= tau", "reached = cum > tau"),
+    "CDF count off by one":
+        ("first = np.argmax(reached, axis=-1) + 1", "first = np.argmax(reached, axis=-1)"),
+    "CDF over ascending probabilities":
+        ('order = np.argsort(-p, axis=-1, kind="stable")', 'order = np.argsort(p, axis=-1, kind="stable")'),
     "a causal mask over the kept tokens":
         ("s = (q_blk @ keys.T) / math.sqrt(d)\n    m = s.max",
          "s = (q_blk @ keys.T) / math.sqrt(d)\n    s = s + np.triu(np.full(s.shape, -np.inf), 1)\n    m = s.max"),

@@ -161,6 +161,71 @@ def test_topk_with_many_ties_matches_brute_force():
             assert list(got) == _brute_force_topk(row, kk)
 
 
+def test_cdf_threshold_closed_forms_on_dyadic_rows():
+    # Exact dyadic probabilities: every partial sum is exact, so "reaches"
+    # (>=) and "exceeds" (>) differ visibly when tau equals a partial sum.
+    row = np.array([0.125, 0.5, 0.0625, 0.25, 0.0625])[None, None, :]
+    assert oracle.cdf_counts(row, 0.5)[0, 0] == 1       # the largest alone reaches 0.5
+    assert oracle.cdf_counts(row, 0.75)[0, 0] == 2      # 0.5 + 0.25
+    assert oracle.cdf_counts(row, 0.7500001)[0, 0] == 3
+    assert oracle.cdf_counts(row, 0.1)[0, 0] == 1       # tau below the maximum
+    assert oracle.cdf_counts(row, 1.0)[0, 0] == 5       # the whole row
+    assert oracle.cdf_counts(row, 2.0)[0, 0] == 5       # never reached: every block
+
+
+def test_cdf_threshold_on_uniform_rows_is_ceil_tau_nb():
+    for nb in (7, 8, 50):
+        row = np.full((1, 1, nb), 1.0 / nb)
+        for tau in (0.13, 0.5, 0.61, 0.97):
+            assert oracle.cdf_counts(row, tau)[0, 0] == math.ceil(tau * nb - 1e-9)
+
+
+def _brute_force_cdf(row, tau):
+    """Smallest subset reaching mass tau; among those, the largest mass, then
+    the lexicographically smallest ascending tuple."""
+    n = len(row)
+    for m in range(1, n + 1):
+        best, best_sum = None, -1.0
+        for comb in itertools.combinations(range(n), m):
+            s = float(sum(row[j] for j in comb))
+            if s >= tau and s > best_sum:
+                best, best_sum = comb, s
+        if best is not None:
+            return m, list(best)
+    return n, list(range(n))
+
+
+def test_cdf_selection_equals_brute_force_on_tiny():
+    w, q, k, v = _tiny_inputs()
+    for tau in (0.3, 0.55, 0.8, 0.95):
+        counts, idx, sc = oracle.select_blocks_cdf(q, k, w.block, tau, w.n_blocks,
+                                                   return_scores=True)
+        assert idx.shape == (w.heads, w.n_blocks, w.n_blocks)
+        for h in range(w.heads):
+            for i in range(w.n_blocks):
+                m, kept = _brute_force_cdf(sc["probs"][h, i], tau)
+                assert counts[h, i] == m
+                assert list(idx[h, i, :m]) == kept
+                assert (idx[h, i, m:] == kept[-1]).all()
+
+
+def test_cdf_counts_grow_with_tau_and_capacity_truncates_to_the_top_blocks():
+    w, q, k, v = _tiny_inputs()
+    probs = oracle.selection_scores(q, k, None, w.block, 0.0)["probs"]
+    prev = np.zeros(probs.shape[:2], dtype=np.int32)
+    for tau in np.linspace(0.05, 1.0, 20):
+        c = oracle.cdf_counts(probs, float(tau))
+        assert (c >= prev).all() and (c >= 1).all() and (c <= w.n_blocks).all()
+        prev = c
+    for tau in (0.3, 0.99):
+        counts, idx = oracle.select_blocks_cdf(q, k, w.block, tau, 2)
+        for h in range(w.heads):
+            for i in range(w.n_blocks):
+                keep = min(2, int(counts[h, i]))
+                kept = sorted(np.argsort(-probs[h, i], kind="stable")[:keep].tolist())
+                assert list(idx[h, i]) == kept + [kept[-1]] * (2 - keep)
+
+
 def test_topk_duplicated_key_block_keeps_lower_index():
     # Block 6 is a copy of block 2, so their pooled scores are bitwise equal.
     rng = np.random.default_rng(17)
