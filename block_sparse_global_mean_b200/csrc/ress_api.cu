@@ -169,6 +169,26 @@ ress_status ress_select_blocks(const ress_shape* shape, const void* q, const voi
                        static_cast<cudaStream_t>(stream));
 }
 
+ress_status ress_select_blocks_cdf(const ress_shape* shape, const void* q, const void* k,
+                                   float tau, int32_t capacity, int32_t* counts, int32_t* idx,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+  Geometry g;
+  ress_status s = check_shape(shape, &g);
+  if (s != RESS_OK) return s;
+  if (!(tau > 0.f && tau <= 1.f)) return RESS_ERR_INVALID_ARG;
+  if ((s = check_budget(g, capacity)) != RESS_OK) return s;
+  if (g.nb == 0) return RESS_OK;
+  if (g.nb > kMaxBlocksSelect) return RESS_ERR_UNSUPPORTED;
+  if (!q || !k || !counts || !idx || !workspace) return RESS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(counts) & 3u))
+    return RESS_ERR_INVALID_ARG;
+  if (workspace_bytes < select_layout(g, false).total) return RESS_ERR_WORKSPACE;
+  const CdfSelect cdf{tau, counts};
+  return launch_select(g, q, k, nullptr, capacity, 0.f, idx, workspace,
+                       static_cast<cudaStream_t>(stream), &cdf);
+}
+
 size_t ress_attn_workspace_bytes(const ress_shape* shape) {
   Geometry g;
   if (check_shape(shape, &g) != RESS_OK) return 0;

@@ -46,8 +46,16 @@ struct DeviceError;
 DeviceError* device_error_ptr();
 
 // Launchers (argument checks are done by the caller).
+// CDF-threshold selection: per row, the count of top blocks whose pooled
+// probabilities reach tau goes to counts[H][nb]; idx rows hold the top
+// min(count, budget) blocks, padded with the last kept block.
+struct CdfSelect {
+  float tau;
+  int32_t* counts;
+};
 ress_status launch_select(const Geometry& g, const void* q, const void* k, const void* v,
-                          int budget, float lambda, int32_t* idx, void* ws, cudaStream_t st);
+                          int budget, float lambda, int32_t* idx, void* ws, cudaStream_t st,
+                          const CdfSelect* cdf = nullptr);
 ress_status launch_attn(const Geometry& g, const void* q, const void* k, const void* v,
                         int budget, const int32_t* idx, void* out, bool out_f32, float* lse,
                         cudaStream_t st);

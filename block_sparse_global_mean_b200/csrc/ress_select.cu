@@ -147,6 +147,8 @@ struct ScoreArgs {
   int row_stride;         // floats between score rows in shared memory
   int stages;             // ring stages
   float lambda;
+  float tau;              // CDF threshold (cdf_counts != null)
+  int32_t* cdf_counts;    // [H][nb] CDF counts, or null for the fixed budget
 };
 
 // Exact selection of `budget` largest keys of a shared-memory row (one warp):
@@ -222,6 +224,12 @@ constexpr int kBins = 512;        // histogram bins, linear in the value over [r
 constexpr int kMaxCand = 64;      // values of the threshold bin that are ranked exactly
 constexpr int kBitmapWords = 128; // kept-block bitmap: nb <= 4096
 constexpr int kWarpScratchWords = kBins + kBitmapWords + 2 * kMaxCand;
+constexpr int kCdfBins = 256;     // histogram bins of the CDF count
+// Per-row-warp scratch: the top-k (kWarpScratchWords) or the CDF count
+// (counts, 64-bit masses and candidates of kCdfBins bins).
+constexpr int kWarpScratchStride = 1024;
+static_assert(kWarpScratchWords <= kWarpScratchStride &&
+              kCdfBins + 2 * kCdfBins + 4 * kMaxCand <= kWarpScratchStride, "row-warp scratch");
 
 // Shared-memory histogram increment; the result is not returned.
 __device__ __forceinline__ void red_add_shared(uint32_t addr, uint32_t v) {
@@ -235,6 +243,13 @@ __device__ __forceinline__ uint32_t value_bin(float v, float lo, float scale) {
   const float d = fmaxf(v - lo, 0.f);
   const uint32_t b = __float_as_uint(fmaf(d, scale, 12582912.0f)) - 0x4B400000u;
   return min(b, (uint32_t)(kBins - 1));
+}
+
+// The same with `bins` bins (scale = (bins - 1) / range).
+__device__ __forceinline__ uint32_t value_bin_n(float v, float lo, float scale, uint32_t bins) {
+  const float d = fmaxf(v - lo, 0.f);
+  const uint32_t b = __float_as_uint(fmaf(d, scale, 12582912.0f)) - 0x4B400000u;
+  return min(b, bins - 1u);
 }
 
 // Exact top-`budget` of a shared-memory row (one warp), lowest index on ties.
@@ -408,6 +423,235 @@ __device__ __forceinline__ void warp_topk_row_binned(const float* row, int nb, i
   }
 }
 
+// Probability of logit s in units of 2^-40: p = exp(s - hi) / z in float32,
+// rounded to the nearest unit.  Sums of up to 4,096 of them are exact in 64
+// bits, so every mass below is independent of the summation order.
+__device__ __forceinline__ unsigned long long mass_fixed(float s, float hi, float inv_z) {
+  return __float2ull_rn(expf(s - hi) * inv_z * 1099511627776.0f);
+}
+
+__device__ __forceinline__ unsigned long long shfl_up_u64(unsigned long long v, int o) {
+  return __shfl_up_sync(0xffffffffu, v, o);
+}
+
+// CDF count of one shared-memory row of pooled logits (one warp): the
+// smallest m >= 1 such that the m largest probabilities (equal logits in
+// index order) sum to at least tau_f (units of 2^-40); nb if the total does
+// not reach it.  Probabilities follow the logits, so logits are ranked.
+//  1. row max hi, z = sum exp(s - hi), and the total mass;
+//  2. over the current logit interval [a, b] (first the whole row): counts
+//     and masses in kCdfBins value-linear bins; the bin b* where the mass
+//     from the top reaches tau_f; the blocks above b* are kept;
+//  3. if b* holds at most kMaxCand blocks, they are ranked exactly by (logit
+//     desc, index asc) and taken in that order until the mass reaches tau_f;
+//     if its blocks all have one logit, the count follows by division;
+//     otherwise [a, b] becomes the logit range of b* and step 2 repeats.
+// Each level separates the distinct logits of b* by a factor of about
+// kCdfBins, so four levels suffice for float32; after six the remaining
+// blocks are taken one at a time in rank order (never reached in practice).
+__device__ __noinline__ int warp_cdf_count(const float* row, int nb, unsigned long long tau_f,
+                                           uint32_t* scratch, int lane) {
+  uint32_t* cnt = scratch;                                                      // [kCdfBins]
+  unsigned long long* mass = reinterpret_cast<unsigned long long*>(scratch + kCdfBins);  // [kCdfBins]
+  uint32_t* ckey = scratch + 3 * kCdfBins;                                      // [kMaxCand]
+  uint32_t* cj = ckey + kMaxCand;                                               // [kMaxCand]
+  unsigned long long* cm = reinterpret_cast<unsigned long long*>(cj + kMaxCand);  // [kMaxCand]
+  const uint32_t lt_mask = (1u << lane) - 1u;
+  const int run = 4 * ((((nb + 31) >> 5) + 3) >> 2 | 1);
+  const int j0 = min(lane * run, nb);
+  const int j1 = min(j0 + run, nb);
+
+  float lo = INFINITY, hi = -INFINITY;
+  for (int j = j0; j < j1; ++j) {
+    lo = fminf(lo, row[j]);
+    hi = fmaxf(hi, row[j]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  float z = 0.f;
+  for (int j = j0; j < j1; ++j) z += expf(row[j] - hi);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  const float inv_z = 1.0f / z;
+  unsigned long long tot = 0ull;
+  for (int j = j0; j < j1; ++j) tot += mass_fixed(row[j], hi, inv_z);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+  if (!(hi >= lo) || tot < tau_f) return nb;   // never reached (or no finite logit)
+
+  float a = lo, b = hi;
+  int cnt_above = 0;                // blocks above the interval, all kept
+  unsigned long long cum_above = 0; // and their mass
+  for (int level = 0; level < 6; ++level) {
+    float scale = (float)(kCdfBins - 1) / (b - a);
+    if (!(scale < INFINITY)) scale = 0.f;
+    for (int t = lane; t < kCdfBins; t += 32) {
+      cnt[t] = 0u;
+      mass[t] = 0ull;
+    }
+    __syncwarp();
+    for (int j = j0; j < j1; ++j) {
+      const float sv = row[j];
+      if (sv >= a && sv <= b) {
+        const uint32_t bin = value_bin_n(sv, a, scale, kCdfBins);
+        atomicAdd(&cnt[bin], 1u);
+        atomicAdd(&mass[bin], mass_fixed(sv, hi, inv_z));
+      }
+    }
+    __syncwarp();
+    // Lane l owns bins kCdfBins-1-8l .. kCdfBins-8-8l (descending).
+    constexpr int kPer = kCdfBins / 32;
+    unsigned long long lm[kPer];
+    int lc[kPer];
+    unsigned long long tm = 0ull;
+    int tc = 0;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      lm[u] = mass[kCdfBins - 1 - kPer * lane - u];
+      lc[u] = (int)cnt[kCdfBins - 1 - kPer * lane - u];
+      tm += lm[u];
+      tc += lc[u];
+    }
+    unsigned long long im = tm;
+    int ic = tc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long ym = shfl_up_u64(im, o);
+      const int yc = __shfl_up_sync(0xffffffffu, ic, o);
+      if (lane >= o) {
+        im += ym;
+        ic += yc;
+      }
+    }
+    const unsigned long long em = im - tm;
+    const int ec = ic - tc;
+    const unsigned ball =
+        __ballot_sync(0xffffffffu, cum_above + em < tau_f && cum_above + im >= tau_f);
+    if (ball == 0u) return nb;      // unreachable: the interval's mass reaches tau_f
+    const int src = __ffs(ball) - 1;
+    int bstar_i = 0, above_c = 0;
+    unsigned long long above_m = 0ull;
+    if (lane == src) {
+      unsigned long long accm = cum_above + em;
+      int accc = ec;
+#pragma unroll
+      for (int u = 0; u < kPer; ++u) {
+        if (accm + lm[u] >= tau_f) {
+          bstar_i = kCdfBins - 1 - kPer * lane - u;
+          above_m = accm;
+          above_c = accc;
+          break;
+        }
+        accm += lm[u];
+        accc += lc[u];
+      }
+    }
+    const uint32_t bstar = (uint32_t)__shfl_sync(0xffffffffu, bstar_i, src);
+    above_c = __shfl_sync(0xffffffffu, above_c, src);
+    above_m = __shfl_sync(0xffffffffu, above_m, src);
+    cnt_above += above_c;
+    cum_above = above_m;
+    const int in_bin = (int)cnt[bstar];
+    if (in_bin <= kMaxCand) {
+      // Gather b* in ascending index order, rank exactly, take in rank order.
+      int n = 0;
+      for (int c0 = 0; c0 < nb; c0 += 32) {
+        const int j = c0 + lane;
+        const float sv = row[min(j, nb - 1)];
+        const bool c = j < nb && sv >= a && sv <= b && value_bin_n(sv, a, scale, kCdfBins) == bstar;
+        const unsigned m = __ballot_sync(0xffffffffu, c);
+        if (c) {
+          const int slot = n + __popc(m & lt_mask);
+          ckey[slot] = order_key(sv);
+          cj[slot] = (uint32_t)j;
+          cm[slot] = mass_fixed(sv, hi, inv_z);
+        }
+        n += __popc(m);
+      }
+      __syncwarp();
+      int best = in_bin;
+      for (int c = lane; c < in_bin; c += 32) {
+        const uint32_t kc = ckey[c], jc = cj[c];
+        int rank = 0;
+        unsigned long long upto = cm[c];
+        for (int o = 0; o < in_bin; ++o) {
+          const bool before = ckey[o] > kc || (ckey[o] == kc && cj[o] < jc);
+          rank += before ? 1 : 0;
+          upto += before ? cm[o] : 0ull;
+        }
+        if (cum_above + upto >= tau_f) best = min(best, rank);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
+      return cnt_above + min(best + 1, in_bin);
+    }
+    // Crowded b*: its logit range becomes the next interval.
+    float na = INFINITY, nbv = -INFINITY;
+    for (int j = j0; j < j1; ++j) {
+      const float sv = row[j];
+      if (sv >= a && sv <= b && value_bin_n(sv, a, scale, kCdfBins) == bstar) {
+        na = fminf(na, sv);
+        nbv = fmaxf(nbv, sv);
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      na = fminf(na, __shfl_xor_sync(0xffffffffu, na, o));
+      nbv = fmaxf(nbv, __shfl_xor_sync(0xffffffffu, nbv, o));
+    }
+    if (na == nbv) {
+      // One logit: every block of b* carries the same mass.
+      const unsigned long long pm = mass_fixed(na, hi, inv_z);
+      const unsigned long long need = tau_f - cum_above;
+      const unsigned long long take = pm ? (need + pm - 1ull) / pm : (unsigned long long)in_bin;
+      return cnt_above + (int)min(take, (unsigned long long)in_bin);
+    }
+    a = na;
+    b = nbv;
+    __syncwarp();
+  }
+  // Last resort: take the blocks of [a, b] one at a time in rank order.
+  uint32_t prev_key = 0xffffffffu;
+  int prev_j = -1;
+  bool first = true;
+  unsigned long long cum = cum_above;
+  int taken = 0;
+  for (int guard = 0; guard < nb; ++guard) {
+    uint32_t bk = 0u;
+    int bj = nb;
+    for (int j = j0; j < j1; ++j) {
+      const float sv = row[j];
+      if (!(sv >= a && sv <= b)) continue;
+      const uint32_t kk = order_key(sv);
+      const bool after = first || kk < prev_key || (kk == prev_key && j > prev_j);
+      if (after && (kk > bk || (kk == bk && j < bj) || bj == nb)) {
+        bk = kk;
+        bj = j;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const uint32_t ok2 = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+      if (oj != nb && (bj == nb || ok2 > bk || (ok2 == bk && oj < bj))) {
+        bk = ok2;
+        bj = oj;
+      }
+    }
+    if (bj == nb) break;
+    ++taken;
+    cum += mass_fixed(row[bj], hi, inv_z);
+    if (cum >= tau_f) break;
+    prev_key = bk;
+    prev_j = bj;
+    first = false;
+  }
+  return cnt_above + max(taken, 1);
+}
+
 // CTA = one head and R consecutive query blocks.  The pooled keys stream
 // through a ring of 16 KB shared-memory stages, each [4 d][1024 keys] fp32,
 // filled by bulk copies that the producer (the last warp) issues as soon as
@@ -430,8 +674,8 @@ struct ScoreCfg {
   static constexpr int kProducer = kWarps - 1;
   // The top-k scratch of the R row warps reuses the stage ring, which has at
   // least 4 stages for R = 16 and 2 for R = 8.
-  static_assert(R * kWarpScratchWords * 4 <= (R == 16 ? 4 : 2) * (int)kStageBytes,
-                "top-k scratch fits the stage ring");
+  static_assert(R * kWarpScratchStride * 4 <= (R == 16 ? 4 : 2) * (int)kStageBytes,
+                "row-warp scratch fits the stage ring");
 };
 
 // Registers are capped at 128 so that four warps of one SM sub-partition fit
@@ -572,8 +816,24 @@ __global__ void __maxnreg__(128) score_topk_kernel(const ScoreArgs a) {
   // One warp per row; the stage buffers now hold each warp's top-k scratch.
   const int i = i0 + warp;
   if (i >= nb) return;
-  uint32_t* whist = reinterpret_cast<uint32_t*>(stages) + warp * kWarpScratchWords;
+  uint32_t* whist = reinterpret_cast<uint32_t*>(stages) + warp * kWarpScratchStride;
   float* row = scores + (size_t)warp * rs;
+  int32_t* out = a.idx + ((size_t)h * nb + i) * a.budget;
+  if (a.cdf_counts != nullptr) {
+    // CDF threshold: the count, then the exact top min(count, capacity) of the
+    // logits (the probabilities' order), padded with the last kept block.
+    // At least one unit: every row keeps at least its top block.
+    const unsigned long long tau_f = max(__double2ull_rn((double)a.tau * 1099511627776.0), 1ull);
+    const int k = warp_cdf_count(row, nb, tau_f, whist, lane);
+    const int keep = min(k, a.budget);
+    __syncwarp();
+    warp_topk_row_binned(row, nb, keep, whist, out, lane);
+    __syncwarp();
+    const int32_t last = out[keep - 1];
+    for (int r = keep + lane; r < a.budget; r += 32) out[r] = last;
+    if (lane == 0) a.cdf_counts[(size_t)h * nb + i] = k;
+    return;
+  }
   if (a.lambda != 0.f) {
     float m = -INFINITY;
     for (int j = lane; j < nb; j += 32) m = fmaxf(m, row[j]);
@@ -587,7 +847,7 @@ __global__ void __maxnreg__(128) score_topk_kernel(const ScoreArgs a) {
     for (int j = lane; j < nb; j += 32) row[j] = expf(row[j] - m) / z + a.lambda * ch[j];
     __syncwarp();
   }
-  warp_topk_row_binned(row, nb, a.budget, whist, a.idx + ((size_t)h * nb + i) * a.budget, lane);
+  warp_topk_row_binned(row, nb, a.budget, whist, out, lane);
 }
 
 // Shared memory of score_topk_kernel<R> with `stages` ring stages and score
@@ -645,7 +905,8 @@ SelectLayout select_layout(const Geometry& g, bool with_v) {
 }
 
 ress_status launch_select(const Geometry& g, const void* q, const void* k, const void* v,
-                          int budget, float lambda, int32_t* idx, void* ws, cudaStream_t st) {
+                          int budget, float lambda, int32_t* idx, void* ws, cudaStream_t st,
+                          const CdfSelect* cdf) {
   const bool with_v = lambda != 0.f;
   const SelectLayout lay = select_layout(g, with_v);
   uint8_t* w = static_cast<uint8_t*>(ws);
@@ -690,6 +951,8 @@ ress_status launch_select(const Geometry& g, const void* q, const void* k, const
   sa.nb_pad = g.nb_pad;
   sa.budget = budget;
   sa.lambda = lambda;
+  sa.tau = cdf ? cdf->tau : 0.f;
+  sa.cdf_counts = cdf ? cdf->counts : nullptr;
   sa.row_stride = (g.nb + 3) & ~3;
   // Sixteen rows per CTA while at least four stages fit next to the score rows
   // (nb <= 2,304), else eight.  The stage ring also holds the top-k scratch of

@@ -63,6 +63,9 @@ lib.ress_block_drift.argtypes = [_SHAPE, _P, _P, _P, ctypes.c_int32, _P, _P, _P,
                                  ctypes.c_size_t, _P]
 lib.ress_select_blocks_noalloc.restype = ctypes.c_int
 lib.ress_select_blocks_noalloc.argtypes = [_SHAPE, _P, _P, _P, ctypes.c_int32, ctypes.c_float, _P, _P]
+lib.ress_select_blocks_cdf.restype = ctypes.c_int
+lib.ress_select_blocks_cdf.argtypes = [_SHAPE, _P, _P, ctypes.c_float, ctypes.c_int32, _P, _P, _P,
+                                         ctypes.c_size_t, _P]
 lib.ress_last_cuda_error.restype = ctypes.c_char_p
 lib.ress_last_cuda_error.argtypes = []
 lib.ress_test_exp2.restype = ctypes.c_int
@@ -145,6 +148,32 @@ def ress_select_blocks(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tenso
                                     workspace.numel(), _stream_ptr(stream, q.device))
     _check(status, "ress_select_blocks")
     return idx
+
+
+def ress_select_blocks_cdf(q: torch.Tensor, k: torch.Tensor, tau: float, block: int,
+                           capacity: Optional[int] = None, counts: Optional[torch.Tensor] = None,
+                           idx: Optional[torch.Tensor] = None,
+                           workspace: Optional[torch.Tensor] = None,
+                           stream: Optional[torch.cuda.Stream] = None
+                           ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Stage 1 with the cumulative (CDF) threshold: returns (counts [H, nb]
+    int32, idx [H, nb, capacity] int32); capacity defaults to nb."""
+    sh = _shape_of(q, block)
+    n, h = q.shape[0], q.shape[1]
+    nb = n // block
+    cap = nb if capacity is None else int(capacity)
+    if counts is None:
+        counts = torch.empty((h, nb), dtype=torch.int32, device=q.device)
+    if idx is None:
+        idx = torch.empty((h, nb, max(cap, 1)), dtype=torch.int32, device=q.device)
+    need = int(lib.ress_select_workspace_bytes(ctypes.byref(sh), ctypes.c_float(0.0)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    status = lib.ress_select_blocks_cdf(ctypes.byref(sh), _ptr(q), _ptr(k), ctypes.c_float(tau),
+                                        cap, _ptr(counts), _ptr(idx), _ptr(workspace),
+                                        workspace.numel(), _stream_ptr(stream, q.device))
+    _check(status, "ress_select_blocks_cdf")
+    return counts, idx
 
 
 def ress_select_blocks_noalloc(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor],

@@ -11,6 +11,9 @@
  *   2. ress_block_sparse_attn  attention restricted to the kept key blocks.
  *   3. ress_block_drift        per-dropped-block drift norm and drop-set drift.
  *
+ * ress_select_blocks_cdf is the SparseVGGT variant of stage 1: a per-row
+ * cumulative probability threshold instead of a fixed budget.
+ *
  * Sources: ReSS: Residual-Restoring Sparse Attention for 3D Vision Transformers
  * (thelatestinai.com) - Abstract, Fig. 1, Fig. 3, Table 1, Table S5, Table S6;
  * VASC: Value-Aware Sparse Attention with Cross-Layer Memory (paperlayer.ai) -
@@ -138,6 +141,36 @@ ress_status ress_select_blocks(const ress_shape* shape, const void* q, const voi
 ress_status ress_select_blocks_noalloc(const ress_shape* shape, const void* q, const void* k,
                                        const void* v, int32_t budget, float lambda,
                                        int32_t* idx, void* stream);
+
+/*
+ * Stage 1 with the cumulative (CDF) threshold of SparseVGGT instead of a fixed
+ * budget (ReSS Table S5: with the similarity gate off, selection is a
+ * cumulative threshold on pooled query/key inner products; ReSS Table 2, row
+ * "+ CDF threshold").  For each head h and query block i, with p_ij the pooled
+ * probabilities of ress_select_blocks (lambda = 0), the count is the smallest
+ * m >= 1 such that the m blocks of largest p (equal values in index order) sum
+ * to at least tau, or nb if the total never reaches tau.
+ *
+ *   q, k       as for ress_select_blocks (no V: the rule has no contrast term).
+ *   tau        0 < tau <= 1.
+ *   capacity   1 <= capacity <= nb: the length of every idx row.
+ *   counts     out, [H][nb] int32: the count of every row (it may exceed
+ *              capacity).
+ *   idx        out, [H][nb][capacity] int32: the top min(count, capacity)
+ *              blocks of the row in ascending order, then the last of them
+ *              repeated to the end of the row, so that idx with
+ *              budget = capacity is a valid kept list for
+ *              ress_block_sparse_attn (duplicates count once there).
+ *   workspace  ress_select_workspace_bytes(shape, 0) bytes, 256-byte aligned.
+ *   Supported sizes: nb <= 4096.
+ *   The probabilities are float32 and their running sum is exact (fixed point
+ *   in units of 2^-40, independent of the summation order), so the result is
+ *   deterministic, and a count can differ from an evaluation in float64 only
+ *   where the cumulative mass lies within about 1e-6 of tau.
+ */
+ress_status ress_select_blocks_cdf(const ress_shape* shape, const void* q, const void* k,
+                                   float tau, int32_t capacity, int32_t* counts, int32_t* idx,
+                                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Workspace bytes that ress_block_sparse_attn and ress_block_drift need:

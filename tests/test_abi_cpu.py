@@ -135,3 +135,27 @@ def test_workspace_queries(ress):
     assert ress.attn_workspace_bytes(n, h, 64, torch.bfloat16) == 0
     assert ress.attn_workspace_bytes(512, 2, 64, torch.float32) == 3 * 512 * 2 * 64 * 2
     assert ress.lib.ress_select_workspace_bytes(None, ctypes.c_float(0.0)) == 0
+
+
+def _cdf(ress, shape, q=FAKE, k=FAKE, tau=0.9, cap=4, counts=FAKE, idx=FAKE, ws=FAKE_WS,
+         ws_bytes=1 << 30):
+    return ress.lib.ress_select_blocks_cdf(ctypes.byref(shape) if shape is not None else None, q,
+                                           k, ctypes.c_float(tau), cap, counts, idx, ws, ws_bytes,
+                                           None)
+
+
+def test_cdf_select_rejects_bad_arguments_on_the_host(ress):
+    E = ress
+    assert _cdf(ress, None) == E.RESS_ERR_INVALID_ARG
+    assert _cdf(ress, _shape(ress, d=32)) == E.RESS_ERR_UNSUPPORTED
+    for tau in (0.0, -0.5, 1.5, float("nan"), float("inf")):
+        assert _cdf(ress, _shape(ress), tau=tau) == E.RESS_ERR_INVALID_ARG, tau
+    assert _cdf(ress, _shape(ress), cap=0) == E.RESS_ERR_INVALID_ARG
+    assert _cdf(ress, _shape(ress), cap=9) == E.RESS_ERR_INVALID_ARG      # nb = 8
+    assert _cdf(ress, _shape(ress), counts=None) == E.RESS_ERR_INVALID_ARG
+    assert _cdf(ress, _shape(ress), counts=FAKE + 2) == E.RESS_ERR_INVALID_ARG
+    assert _cdf(ress, _shape(ress), idx=None) == E.RESS_ERR_INVALID_ARG
+    assert _cdf(ress, _shape(ress), q=FAKE + 8) == E.RESS_ERR_INVALID_ARG
+    assert _cdf(ress, _shape(ress), ws_bytes=16) == E.RESS_ERR_WORKSPACE
+    assert _cdf(ress, _shape(ress, n=64 * 4097), cap=1) == E.RESS_ERR_UNSUPPORTED
+    assert _cdf(ress, _shape(ress, n=0), cap=0) == E.RESS_OK               # empty: no launch
