@@ -10,10 +10,15 @@
 //                      whose few values are ranked exactly) that keeps
 //                      `budget` blocks, ties to the lower index, written in
 //                      ascending order.
+//                      In its CDF mode each row keeps instead the fewest top
+//                      blocks whose probabilities reach tau (warp_cdf_count),
+//                      padded to a fixed capacity.
 //
 // Sources: ReSS (thelatestinai.com) Table S5, SpargeAttn row - selection by
-// pooled query/key inner products; VASC (paperlayer.ai) 4.1 - pooled relevance
-// plus neighbouring value contrast; VASC A.2 - an exact-capacity binary Top-K.
+// pooled query/key inner products, which reduces to SparseVGGT's cumulative
+// threshold (Table 2, "+ CDF threshold"); VASC (paperlayer.ai) 4.1 - pooled
+// relevance plus neighbouring value contrast; VASC A.2 - an exact-capacity
+// binary Top-K.
 #include "ress_common.cuh"
 #include "ress_internal.h"
 
