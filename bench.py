@@ -40,6 +40,22 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 KERNEL_SOURCES = ["ress_attn.cu", "ress_common.cuh"]
 
 
+def input_bytes(w) -> int:
+    """Q + K + V bytes one step reads."""
+    elem = 2 if w.dtype == "bf16" else 4
+    return 3 * w.n_tokens * w.heads * w.head_dim * elem
+
+
+def l2_policy(w):
+    """(flush, description): inputs under twice the L2 size are timed with an
+    L2 flush (a 256 MB write) before every timed step, outside its events."""
+    mb = input_bytes(w) / 1e6
+    if input_bytes(w) >= 2 * L2_BYTES:
+        return False, "inputs larger than L2 (Q+K+V = %.0f MB per step)" % mb
+    return True, "L2 flushed before every timed step by a 256 MB write outside the timed events " \
+                 "(Q+K+V = %.1f MB per step)" % mb
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -169,7 +185,7 @@ def workload_config(w, world: int):
         "global_batch": world,
         "tokens_per_rank": w.n_tokens,
         "step": "select(pool+score+topk) -> block-sparse attention" + (" -> drift" if w.drift else ""),
-        "l2": "inputs larger than L2 (Q+K+V = %.0f MB per step)" % (3 * w.n_tokens * w.heads * 64 * 2 / 1e6),
+        "l2": l2_policy(w)[1],
         "parallelism": f"dp{world} (independent inputs per rank)",
     }
 
@@ -311,15 +327,24 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize(dev)
+    flush, _ = l2_policy(w)
+    scratch = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush else None
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
-    for _ in range(args.steps):
+    for it in range(args.steps):
+        if flush:
+            scratch.fill_(it & 255)
         step(q, k, v, record=True)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
-    elapsed_ms = t_start.elapsed_time(t_end)
+    if flush:
+        # Each step from its first to its last event; the flushes lie between.
+        last = ev["dr1"] if w.drift else ev["att1"]
+        elapsed_ms = sum(a.elapsed_time(b) for a, b in zip(ev["sel0"], last))
+    else:
+        elapsed_ms = t_start.elapsed_time(t_end)
 
     def mean_pair(a, b):
         return sum(x.elapsed_time(y) for x, y in zip(ev[a], ev[b])) / max(1, len(ev[a]))
