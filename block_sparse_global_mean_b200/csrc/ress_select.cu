@@ -818,7 +818,7 @@ __global__ void __maxnreg__(128) score_topk_kernel(const ScoreArgs a) {
   }
   __syncthreads();
   if (*abortf != 0 || warp >= R) return;
-  // One warp per row; the stage buffers now hold each warp's top-k scratch.
+  // One warp per row; the stage buffers now hold each row warp's scratch.
   const int i = i0 + warp;
   if (i >= nb) return;
   uint32_t* whist = reinterpret_cast<uint32_t*>(stages) + warp * kWarpScratchStride;
