@@ -33,6 +33,13 @@ Readings taken where the pages are silent (each is repeated at its function):
 * the drift contribution of a dropped block uses the kept-set normaliser lse;
   its norm is the Frobenius norm over the block's B x d contribution matrix, and
   the drop-set drift J is the Frobenius norm of the summed contributions.
+* the CDF threshold keeps the fewest top blocks whose probabilities reach tau
+  (ties to the lower index; every block if the total never reaches tau);
+* with padding and special tokens: blocks pool their valid tokens only,
+  padding keys never enter a softmax and padding queries write nothing,
+  special (camera, register) queries attend densely to every valid key,
+  key blocks made only of special tokens are always kept, and special queries
+  drop nothing in the drift.
 
 Every function here is pinned by the tests in ``tests/test_oracle_pins.py``
 against closed forms, brute force, invariants or independent library routines.
@@ -323,3 +330,143 @@ def block_drift(q, k, v, idx, lse, block: int,
         drift[h, i, :] = dr
         jset[h, i] = jv
     return drift, jset
+
+
+# ---------------------------------------------------------------------------
+# Layout-aware variant: padding and the special (camera, register) tokens
+# ---------------------------------------------------------------------------
+
+def view_layout(n_tokens: int, tokens_per_view: int, real_tokens_per_view: int,
+                n_special: int = 5) -> Tuple[np.ndarray, np.ndarray]:
+    """Boolean masks (valid [N], special [N]) of concatenated padded views.
+
+    A VGGT view is 1 camera + 4 register tokens followed by its patch tokens,
+    zero-padded to ``tokens_per_view``; positions ``real_tokens_per_view`` ..
+    ``tokens_per_view - 1`` of every view are padding, positions 0 ..
+    ``n_special - 1`` are the special tokens.
+    """
+    pos = np.arange(n_tokens) % tokens_per_view
+    valid = pos < real_tokens_per_view
+    special = valid & (pos < n_special)
+    return valid, special
+
+
+def pool_blocks_valid(x, block: int, valid) -> Tuple[np.ndarray, np.ndarray]:
+    """Mean of the valid tokens of each block, per head, and the valid counts.
+
+    Reading: padding does not enter a block's mean; a block without a valid
+    token pools to the zero vector and is empty.  Returns (pooled [H, nb, d],
+    counts [nb]).
+    """
+    x = _f64(x)
+    valid = np.asarray(valid, dtype=bool)
+    n, h, d = x.shape
+    nb = n // block
+    w = valid.reshape(nb, block).astype(np.float64)
+    counts = w.sum(axis=1)
+    sums = np.einsum("jb,jbhd->jhd", w, x.reshape(nb, block, h, d))
+    pooled = sums / np.maximum(counts, 1.0)[:, None, None]
+    return np.ascontiguousarray(pooled.transpose(1, 0, 2)), counts.astype(np.int64)
+
+
+def select_blocks_layout(q, k, block: int, budget: int, valid, special,
+                         return_scores: bool = False):
+    """Stage 1 with padding and special tokens (VASC section 4.2: camera and
+    register queries stay dense and key blocks made only of special tokens
+    are always kept; VASC A.5: the special queries keep dense attention).
+
+    Readings: pooled means over valid tokens only; the pooled logits as in
+    ``block_logits``; an empty key block is never preferred to a non-empty
+    one; a special-only key block (at least one valid token, all of them
+    special) is always kept and counts toward the budget (when there are more
+    than ``budget`` of them, the lowest-index ones); the rest of the budget
+    goes to the largest logits, ties to the lower index.
+    """
+    valid = np.asarray(valid, dtype=bool)
+    special = np.asarray(special, dtype=bool)
+    qbar, _ = pool_blocks_valid(q, block, valid)
+    kbar, kcount = pool_blocks_valid(k, block, valid)
+    logits = block_logits(qbar, kbar)
+    nb = kbar.shape[1]
+    sp = (special & valid).reshape(nb, block).sum(axis=1)
+    forced = (kcount > 0) & (sp == kcount)
+    empty = kcount == 0
+    rank = logits.copy()
+    rank[:, :, empty] = -np.inf
+    rank[:, :, forced] = np.inf
+    idx = topk_lowest_index(rank, budget)
+    if return_scores:
+        return idx, {"logits": logits, "forced": forced, "empty": empty}
+    return idx
+
+
+def sparse_attention_layout_block(q, k, v, kept: Sequence[int], h: int, i: int, block: int,
+                                  valid, special) -> Tuple[np.ndarray, np.ndarray]:
+    """Stage 2 for query block ``i`` of head ``h`` with padding and special tokens.
+
+    For query token n: a padding query gets output 0 and lse -inf; a special
+    query attends densely to every valid key of the sequence; any other query
+    attends to the valid tokens of the kept blocks.  Padding keys never enter
+    a softmax.  Returns (O [B, d], lse [B]).
+    """
+    valid = np.asarray(valid, dtype=bool)
+    special = np.asarray(special, dtype=bool)
+    q_h = _f64(q[:, h, :])
+    k_h = _f64(k[:, h, :])
+    v_h = _f64(v[:, h, :])
+    n, d = k_h.shape
+    kept_tok = np.zeros(n, dtype=bool)
+    for j in kept:
+        kept_tok[j * block:(j + 1) * block] = True
+    out = np.zeros((block, d))
+    lse = np.full(block, -np.inf)
+    for r in range(block):
+        t = i * block + r
+        if not valid[t]:
+            continue
+        keys = valid if special[t] else (valid & kept_tok)
+        if not keys.any():
+            continue
+        s = (k_h[keys] @ q_h[t]) / math.sqrt(d)
+        m = s.max()
+        e = np.exp(s - m)
+        out[r] = (e @ v_h[keys]) / e.sum()
+        lse[r] = m + np.log(e.sum())
+    return out, lse
+
+
+def drift_layout_block(q, k, v, kept: Sequence[int], lse_blk, h: int, i: int, block: int,
+                       valid, special) -> Tuple[np.ndarray, float]:
+    """Stage 3 for query block ``i`` of head ``h`` with padding and special tokens.
+
+    As ``drift_block`` over the valid keys of each dropped block, for the
+    valid non-special queries of block i; a special query drops nothing and a
+    padding query writes nothing, so their rows of every C_j are zero.
+    """
+    valid = np.asarray(valid, dtype=bool)
+    special = np.asarray(special, dtype=bool)
+    q_h = _f64(q[:, h, :])
+    k_h = _f64(k[:, h, :])
+    v_h = _f64(v[:, h, :])
+    n, d = k_h.shape
+    nb = n // block
+    lse_blk = _f64(lse_blk)
+    drop = dropped_blocks(kept, nb)
+    if drop.shape[0] == 0:
+        return np.zeros(0), 0.0
+    rows = np.arange(i * block, (i + 1) * block)
+    live = valid[rows] & ~special[rows]
+    contrib = np.zeros((drop.shape[0], block, d))
+    for c, j in enumerate(drop):
+        toks = np.arange(j * block, (j + 1) * block)
+        toks = toks[valid[toks]]
+        if toks.shape[0] == 0:
+            continue
+        s = (q_h[rows] @ k_h[toks].T) / math.sqrt(d)
+        # rows that write nothing (lse -inf for padding) take a finite stand-in
+        lse_live = np.where(live, lse_blk, 0.0)
+        w = np.exp(s - lse_live[:, None]) * live[:, None]
+        contrib[c] = w @ v_h[toks]
+    drift = np.sqrt((contrib * contrib).sum(axis=(1, 2)))
+    total = contrib.sum(axis=0)
+    return drift, float(np.sqrt((total * total).sum()))

@@ -42,6 +42,19 @@ MUTATIONS = {
         ("first = np.argmax(reached, axis=-1) + 1", "first = np.argmax(reached, axis=-1)"),
     "CDF over ascending probabilities":
         ('order = np.argsort(-p, axis=-1, kind="stable")', 'order = np.argsort(p, axis=-1, kind="stable")'),
+    "padding pooled into the block means":
+        ("w = valid.reshape(nb, block).astype(np.float64)", "w = np.ones((nb, block))"),
+    "padding keys enter the softmax":
+        ("keys = valid if special[t] else (valid & kept_tok)",
+         "keys = np.ones(n, dtype=bool) if special[t] else kept_tok"),
+    "special queries follow the sparse mask":
+        ("keys = valid if special[t] else (valid & kept_tok)", "keys = valid & kept_tok"),
+    "special-only key blocks not forced":
+        ("rank[:, :, forced] = np.inf", "rank[:, :, forced] = rank[:, :, forced]"),
+    "special queries counted in the drift":
+        ("live = valid[rows] & ~special[rows]", "live = valid[rows]"),
+    "padding keys in the drift":
+        ("toks = toks[valid[toks]]", "toks = toks"),
     "a causal mask over the kept tokens":
         ("s = (q_blk @ keys.T) / math.sqrt(d)\n    m = s.max",
          "s = (q_blk @ keys.T) / math.sqrt(d)\n    s = s + np.triu(np.full(s.shape, -np.inf), 1)\n    m = s.max"),

@@ -426,3 +426,154 @@ def test_drift_closed_form_with_zero_queries_and_orthogonal_values():
             expect = math.sqrt(B) * abs(col_sum) / (budget * B)
             assert drift[0, i, r] == pytest.approx(expect, rel=1e-12)
         assert jset[0, i] == pytest.approx(math.sqrt((drift[0, i] ** 2).sum()), rel=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Layout-aware variant: padding and special tokens
+# --------------------------------------------------------------------------
+
+def _layout_case(seed=21, views=3, tpv=16, real=13, n_special=2, B=4, H=2, d=16):
+    rng = np.random.default_rng(seed)
+    n = views * tpv
+    q = rng.normal(size=(n, H, d))
+    k = rng.normal(size=(n, H, d))
+    v = rng.normal(size=(n, H, d))
+    valid, special = oracle.view_layout(n, tpv, real, n_special)
+    return q, k, v, valid, special, B
+
+
+def test_layout_reduces_to_the_plain_path_without_padding_or_special_tokens():
+    q, k, v, _, _, B = _layout_case()
+    n = q.shape[0]
+    valid = np.ones(n, dtype=bool)
+    special = np.zeros(n, dtype=bool)
+    nb, budget = n // B, 5
+    idx = oracle.select_blocks_layout(q, k, B, budget, valid, special)
+    assert (idx == oracle.select_blocks(q, k, None, B, budget)).all()
+    for h, i in [(0, 0), (1, 5), (0, nb - 1)]:
+        o, l = oracle.sparse_attention_layout_block(q, k, v, idx[h, i], h, i, B, valid, special)
+        o2, l2 = oracle.sparse_attention_block(q, k, v, idx[h, i], h, i, B)
+        assert np.allclose(o, o2, atol=1e-12) and np.allclose(l, l2, atol=1e-12)
+        dr, jv = oracle.drift_layout_block(q, k, v, idx[h, i], l, h, i, B, valid, special)
+        dr2, jv2 = oracle.drift_block(q, k, v, idx[h, i], l2, h, i, B)
+        assert np.allclose(dr, dr2, atol=1e-12) and abs(jv - jv2) < 1e-12
+
+
+def test_padding_values_change_nothing():
+    q, k, v, valid, special, B = _layout_case()
+    rng = np.random.default_rng(5)
+    q2, k2, v2 = q.copy(), k.copy(), v.copy()
+    pad = ~valid
+    for x in (q2, k2, v2):
+        x[pad] = rng.normal(size=x[pad].shape) * 100.0
+    nb, budget = q.shape[0] // B, 4
+    idx = oracle.select_blocks_layout(q, k, B, budget, valid, special)
+    assert (idx == oracle.select_blocks_layout(q2, k2, B, budget, valid, special)).all()
+    for h in range(q.shape[1]):
+        for i in range(nb):
+            o, l = oracle.sparse_attention_layout_block(q, k, v, idx[h, i], h, i, B, valid, special)
+            o2, l2 = oracle.sparse_attention_layout_block(q2, k2, v2, idx[h, i], h, i, B, valid,
+                                                          special)
+            assert np.allclose(o, o2, atol=1e-12) and np.array_equal(np.isinf(l), np.isinf(l2))
+            dr, jv = oracle.drift_layout_block(q, k, v, idx[h, i], l, h, i, B, valid, special)
+            dr2, jv2 = oracle.drift_layout_block(q2, k2, v2, idx[h, i], l2, h, i, B, valid, special)
+            assert np.allclose(dr, dr2, atol=1e-10) and abs(jv - jv2) < 1e-10
+
+
+def test_special_queries_attend_densely_and_padding_queries_write_nothing():
+    q, k, v, valid, special, B = _layout_case()
+    n, H, d = q.shape
+    idx = oracle.select_blocks_layout(q, k, B, 2, valid, special)
+    for h in range(H):
+        kv = torch.tensor(k[valid, h])[None, None]
+        vv = torch.tensor(v[valid, h])[None, None]
+        for i in range(n // B):
+            o, l = oracle.sparse_attention_layout_block(q, k, v, idx[h, i], h, i, B, valid, special)
+            for r in range(B):
+                t = i * B + r
+                if special[t]:
+                    ref = F.scaled_dot_product_attention(torch.tensor(q[t, h])[None, None, None],
+                                                         kv, vv)[0, 0, 0].numpy()
+                    assert np.allclose(o[r], ref, atol=1e-12)
+                    s = torch.tensor(k[valid, h]) @ torch.tensor(q[t, h]) / math.sqrt(d)
+                    assert abs(l[r] - float(torch.logsumexp(s, 0))) < 1e-12
+                if not valid[t]:
+                    assert (o[r] == 0).all() and l[r] == -np.inf
+
+
+def test_pooling_averages_valid_tokens_only():
+    B, H, d = 8, 2, 4
+    x = np.full((2 * B, H, d), 1e6)                      # padding: huge values
+    x[:5] = 0.375                                        # five valid tokens of block 0
+    x[B:B + 8] = np.arange(8, dtype=float)[:, None, None] / 4.0
+    valid = np.zeros(2 * B, dtype=bool)
+    valid[:5] = True
+    valid[B:] = True
+    pooled, counts = oracle.pool_blocks_valid(x, B, valid)
+    assert list(counts) == [5, 8]
+    assert (pooled[:, 0] == 0.375).all()
+    assert (pooled[:, 1] == 7.0 / 8.0).all()             # mean of 0, 1/4, ..., 7/4
+    empty, c0 = oracle.pool_blocks_valid(x, B, np.zeros(2 * B, dtype=bool))
+    assert (empty == 0).all() and (c0 == 0).all()
+
+
+def test_special_only_key_blocks_are_always_kept():
+    # Blocks of 4 tokens; the first block of every 12-token view holds only
+    # the 4 special tokens.  Their keys point away from every query, so their
+    # logits are the lowest of each row, yet they are kept.
+    rng = np.random.default_rng(31)
+    views, tpv, B, H, d = 3, 12, 4, 1, 8
+    n = views * tpv
+    q = np.abs(rng.normal(size=(n, H, d))) + 1.0
+    k = np.abs(rng.normal(size=(n, H, d))) + 1.0
+    valid, special = oracle.view_layout(n, tpv, tpv, 4)
+    k[special] = -5.0
+    idx, sc = oracle.select_blocks_layout(q, k, B, 4, valid, special, return_scores=True)
+    forced = [j for j in range(n // B) if sc["forced"][j]]
+    assert forced == [0, 3, 6]
+    for i in range(n // B):
+        assert set(forced) <= set(idx[0, i].tolist())
+        assert all(sc["logits"][0, i, j] == sc["logits"][0, i].min() or j not in forced
+                   for j in forced)
+        others = [j for j in idx[0, i].tolist() if j not in forced]
+        rest = [j for j in np.argsort(-sc["logits"][0, i], kind="stable") if j not in forced]
+        assert others == sorted(rest[:1])
+
+
+def test_layout_drift_reconstructs_dense_attention_over_valid_keys():
+    q, k, v, valid, special, B = _layout_case(seed=41)
+    n, H, d = q.shape
+    idx = oracle.select_blocks_layout(q, k, B, 4, valid, special)
+    for h in range(H):
+        for i in range(n // B):
+            o, l = oracle.sparse_attention_layout_block(q, k, v, idx[h, i], h, i, B, valid, special)
+            kept_tok = np.zeros(n, dtype=bool)
+            for j in idx[h, i]:
+                kept_tok[j * B:(j + 1) * B] = True
+            drop_tok = valid & ~kept_tok
+            for r in range(B):
+                t = i * B + r
+                if not valid[t] or special[t]:
+                    continue
+                # dense over the valid keys, from torch only
+                dense = F.scaled_dot_product_attention(
+                    torch.tensor(q[t, h])[None, None, None], torch.tensor(k[valid, h])[None, None],
+                    torch.tensor(v[valid, h])[None, None])[0, 0, 0].numpy()
+                s = (k[drop_tok, h] @ q[t, h]) / math.sqrt(d)
+                w = np.exp(s - l[r])
+                c_sum = w @ v[drop_tok, h]
+                assert np.allclose((o[r] + c_sum) / (1.0 + w.sum()), dense, atol=1e-10)
+            # every C_j row of a special or padding query is zero: a block of
+            # only such queries has zero drift
+            dr, jv = oracle.drift_layout_block(q, k, v, idx[h, i], l, h, i, B, valid, special)
+            rows = np.arange(i * B, (i + 1) * B)
+            if not (valid[rows] & ~special[rows]).any():
+                assert (dr == 0).all() and jv == 0.0
+            else:
+                assert jv <= dr.sum() + 1e-12
+    # a block made only of special queries: zero drift, whatever it drops
+    vq, sq = oracle.view_layout(n, 16, 16, 8)
+    idx2 = oracle.select_blocks_layout(q, k, B, 2, vq, sq)
+    o, l = oracle.sparse_attention_layout_block(q, k, v, idx2[0, 0], 0, 0, B, vq, sq)
+    dr, jv = oracle.drift_layout_block(q, k, v, idx2[0, 0], l, 0, 0, B, vq, sq)
+    assert dr.shape[0] > 0 and (dr == 0).all() and jv == 0.0
