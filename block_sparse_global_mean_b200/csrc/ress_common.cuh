@@ -120,7 +120,7 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, D
 }
 
 // ---------------------------------------------------------------------------
-// TMA (tiled tensor loads, no multicast)
+// TMA (tiled tensor loads; every CTA fetches its own tiles)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
