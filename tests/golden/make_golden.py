@@ -40,6 +40,23 @@ def main():
         "drift_h0_i0": drift[0, 0].tolist(),
         "J": jset.tolist(),
     }
+    # CDF threshold on the same pooled probabilities.
+    for tau in (0.5, 0.9):
+        counts, cidx = oracle.select_blocks_cdf(q, k, w.block, tau, w.n_blocks)
+        fixture[f"cdf_counts_tau{tau}"] = counts.tolist()
+        fixture[f"cdf_idx_tau{tau}"] = cidx.tolist()
+    # Layout-aware variant: 2 views of 256 tokens, the last 20 of each padding,
+    # the first 5 special.
+    valid, special = oracle.view_layout(w.n_tokens, 256, 236, 5)
+    lidx = oracle.select_blocks_layout(q, k, w.block, w.budget, valid, special)
+    fixture["layout_idx"] = lidx.tolist()
+    lo, ll = oracle.sparse_attention_layout_block(q, k, v, lidx[1, 3], 1, 3, w.block, valid, special)
+    fixture["layout_out_h1_i3_rows"] = [0, 4, 5, 63]
+    fixture["layout_out_h1_i3"] = lo[[0, 4, 5, 63]].tolist()
+    fixture["layout_lse_h1_i3"] = [float(x) for x in ll]
+    ld, lj = oracle.drift_layout_block(q, k, v, lidx[1, 3], ll, 1, 3, w.block, valid, special)
+    fixture["layout_drift_h1_i3"] = ld.tolist()
+    fixture["layout_J_h1_i3"] = lj
     with open(os.path.join(HERE, "oracle_tiny.json"), "w") as f:
         json.dump(fixture, f, indent=1)
         f.write("\n")

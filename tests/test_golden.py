@@ -27,3 +27,25 @@ def test_oracle_reproduces_recorded_tiny_outputs():
     drift, jset = oracle.block_drift(q, k, v, idx, lse, w.block)
     np.testing.assert_allclose(drift[0, 0], g["drift_h0_i0"], rtol=1e-12)
     np.testing.assert_allclose(jset, g["J"], rtol=1e-12)
+
+
+def test_oracle_reproduces_recorded_cdf_and_layout_outputs():
+    with open(os.path.join(HERE, "oracle_tiny.json")) as f:
+        g = json.load(f)
+    w = workloads.WORKLOADS["tiny"]
+    q, k, v = (t.to(torch.float64).numpy() for t in workloads.generate(w))
+    for tau in (0.5, 0.9):
+        counts, cidx = oracle.select_blocks_cdf(q, k, w.block, tau, w.n_blocks)
+        np.testing.assert_array_equal(counts, np.array(g[f"cdf_counts_tau{tau}"]))
+        np.testing.assert_array_equal(cidx, np.array(g[f"cdf_idx_tau{tau}"]))
+    valid, special = oracle.view_layout(w.n_tokens, 256, 236, 5)
+    lidx = oracle.select_blocks_layout(q, k, w.block, w.budget, valid, special)
+    np.testing.assert_array_equal(lidx, np.array(g["layout_idx"]))
+    lo, ll = oracle.sparse_attention_layout_block(q, k, v, lidx[1, 3], 1, 3, w.block, valid,
+                                                  special)
+    np.testing.assert_allclose(lo[g["layout_out_h1_i3_rows"]], g["layout_out_h1_i3"],
+                               rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(ll, g["layout_lse_h1_i3"], rtol=1e-12)
+    ld, lj = oracle.drift_layout_block(q, k, v, lidx[1, 3], ll, 1, 3, w.block, valid, special)
+    np.testing.assert_allclose(ld, g["layout_drift_h1_i3"], rtol=1e-12, atol=1e-300)
+    np.testing.assert_allclose(lj, g["layout_J_h1_i3"], rtol=1e-12)
