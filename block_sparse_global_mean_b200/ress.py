@@ -120,6 +120,47 @@ def _shape_of(q: torch.Tensor, block: int) -> ress_shape:
     return make_shape(n, h, block, q.dtype, d)
 
 
+def _check_inputs(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor] = None) -> None:
+    """k and v must match q in shape, dtype and device (the library reads all
+    three with q's shape)."""
+    if q.dim() != 3:
+        raise ValueError("q, k, v must be [N, H, d]")
+    for name, t in (("k", k), ("v", v)):
+        if t is None:
+            continue
+        if tuple(t.shape) != tuple(q.shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, q has {tuple(q.shape)}")
+        if t.dtype != q.dtype:
+            raise TypeError(f"{name} is {t.dtype}, q is {q.dtype}")
+        if t.device != q.device:
+            raise ValueError(f"{name} is on {t.device}, q on {q.device}")
+
+
+def _check_buffer(t: torch.Tensor, shape, dtype: torch.dtype, device: torch.device,
+                  name: str) -> None:
+    """A caller-provided buffer must have exactly the shape, dtype and device
+    the library writes or reads."""
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+
+
+def _check_workspace(ws: Optional[torch.Tensor], device: torch.device) -> None:
+    if ws is not None:
+        _check_buffer(ws, (ws.numel(),), torch.uint8, device, "workspace")
+
+
+def _check_idx(idx: torch.Tensor, h: int, nb: int, device: torch.device) -> int:
+    """idx must be int32 [H, nb, budget]; returns budget."""
+    if idx.dim() != 3:
+        raise ValueError(f"idx must be [H, nb, budget], got {tuple(idx.shape)}")
+    _check_buffer(idx, (h, nb, idx.shape[2]), torch.int32, device, "idx")
+    return int(idx.shape[2])
+
+
 def select_workspace_bytes(n: int, heads: int, block: int, dtype: torch.dtype, lam: float) -> int:
     sh = make_shape(n, heads, block, dtype)
     return int(lib.ress_select_workspace_bytes(ctypes.byref(sh), ctypes.c_float(lam)))
@@ -135,11 +176,14 @@ def ress_select_blocks(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tenso
                        workspace: Optional[torch.Tensor] = None,
                        stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """Stage 1: returns idx [H, nb, budget] int32 (ascending kept blocks per row)."""
+    _check_inputs(q, k, v if lam else None)
     sh = _shape_of(q, block)
     n, h = q.shape[0], q.shape[1]
     nb = n // block
     if idx is None:
         idx = torch.empty((h, nb, budget), dtype=torch.int32, device=q.device)
+    _check_buffer(idx, (h, nb, budget), torch.int32, q.device, "idx")
+    _check_workspace(workspace, q.device)
     need = int(lib.ress_select_workspace_bytes(ctypes.byref(sh), ctypes.c_float(lam)))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
@@ -158,6 +202,7 @@ def ress_select_blocks_cdf(q: torch.Tensor, k: torch.Tensor, tau: float, block: 
                            ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Stage 1 with the cumulative (CDF) threshold: returns (counts [H, nb]
     int32, idx [H, nb, capacity] int32); capacity defaults to nb."""
+    _check_inputs(q, k)
     sh = _shape_of(q, block)
     n, h = q.shape[0], q.shape[1]
     nb = n // block
@@ -166,6 +211,9 @@ def ress_select_blocks_cdf(q: torch.Tensor, k: torch.Tensor, tau: float, block: 
         counts = torch.empty((h, nb), dtype=torch.int32, device=q.device)
     if idx is None:
         idx = torch.empty((h, nb, max(cap, 1)), dtype=torch.int32, device=q.device)
+    _check_buffer(counts, (h, nb), torch.int32, q.device, "counts")
+    _check_buffer(idx, (h, nb, max(cap, 1)), torch.int32, q.device, "idx")
+    _check_workspace(workspace, q.device)
     need = int(lib.ress_select_workspace_bytes(ctypes.byref(sh), ctypes.c_float(0.0)))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
@@ -182,10 +230,12 @@ def ress_select_blocks_noalloc(q: torch.Tensor, k: torch.Tensor, v: Optional[tor
                                stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
     """Stage 1 with the library's fixed scratch array instead of a workspace
     (for callers that cannot allocate device memory); see include/ress.h."""
+    _check_inputs(q, k, v if lam else None)
     sh = _shape_of(q, block)
     n, h = q.shape[0], q.shape[1]
     if idx is None:
         idx = torch.empty((h, n // block, budget), dtype=torch.int32, device=q.device)
+    _check_buffer(idx, (h, n // block, budget), torch.int32, q.device, "idx")
     status = lib.ress_select_blocks_noalloc(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(budget),
                                             ctypes.c_float(lam), _ptr(idx),
                                             _stream_ptr(stream, q.device))
@@ -204,17 +254,22 @@ def ress_block_sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, id
 
     The output dtype is ``out.dtype`` if ``out`` is given, else ``out_dtype``,
     else the input dtype."""
+    _check_inputs(q, k, v)
     sh = _shape_of(q, block)
     n, h = q.shape[0], q.shape[1]
-    budget = idx.shape[-1]
+    budget = _check_idx(idx, h, n // block, q.device)
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
     out_code = RESS_F32 if out.dtype == torch.float32 else (
         RESS_BF16 if out.dtype == torch.bfloat16 else None)
     if out_code is None:
         raise TypeError(f"unsupported output dtype {out.dtype}")
+    _check_buffer(out, q.shape, out.dtype, q.device, "out")
     if lse is None and want_lse:
         lse = torch.empty((h, n), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _check_buffer(lse, (h, n), torch.float32, q.device, "lse")
+    _check_workspace(workspace, q.device)
     need = int(lib.ress_attn_workspace_bytes(ctypes.byref(sh)))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
@@ -233,14 +288,19 @@ def ress_block_drift(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: tor
                      stream: Optional[torch.cuda.Stream] = None
                      ) -> Tuple[torch.Tensor, torch.Tensor]:
     """Stage 3: returns (drift [H, nb, nb - budget], set_drift [H, nb]) float32."""
+    _check_inputs(q, k, v)
     sh = _shape_of(q, block)
     n, h = q.shape[0], q.shape[1]
     nb = n // block
-    budget = idx.shape[-1]
+    budget = _check_idx(idx, h, nb, q.device)
+    _check_buffer(lse, (h, n), torch.float32, q.device, "lse")
     if drift is None:
-        drift = torch.empty((h, nb, nb - budget), dtype=torch.float32, device=q.device)
+        drift = torch.empty((h, nb, max(nb - budget, 0)), dtype=torch.float32, device=q.device)
     if set_drift is None:
         set_drift = torch.empty((h, nb), dtype=torch.float32, device=q.device)
+    _check_buffer(drift, (h, nb, max(nb - budget, 0)), torch.float32, q.device, "drift")
+    _check_buffer(set_drift, (h, nb), torch.float32, q.device, "set_drift")
+    _check_workspace(workspace, q.device)
     need = int(lib.ress_attn_workspace_bytes(ctypes.byref(sh)))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)

@@ -159,3 +159,42 @@ def test_cdf_select_rejects_bad_arguments_on_the_host(ress):
     assert _cdf(ress, _shape(ress), ws_bytes=16) == E.RESS_ERR_WORKSPACE
     assert _cdf(ress, _shape(ress, n=64 * 4097), cap=1) == E.RESS_ERR_UNSUPPORTED
     assert _cdf(ress, _shape(ress, n=0), cap=0) == E.RESS_OK               # empty: no launch
+
+
+def test_binding_rejects_mismatched_tensors_before_any_library_call(ress):
+    """Shapes, dtypes and devices that the kernels would read or write out of
+    bounds are refused by the binding (these checks need no GPU)."""
+    import torch
+    bf = torch.bfloat16
+    H, B, nb = 2, 64, 4
+    q = torch.zeros(nb * B, H, 64, dtype=bf)
+    k_short = torch.zeros((nb - 1) * B, H, 64, dtype=bf)
+    with pytest.raises(ValueError, match="k has shape"):
+        ress.ress_select_blocks(q, k_short, None, 2, 0.0, B)
+    with pytest.raises(TypeError, match="v is"):
+        ress.ress_block_sparse_attn(q, q, q.float(), torch.zeros(H, nb, 2, dtype=torch.int32), B)
+    with pytest.raises(TypeError, match="idx must be"):
+        ress.ress_block_sparse_attn(q, q, q, torch.zeros(H, nb, 2, dtype=torch.int64), B)
+    with pytest.raises(ValueError, match="idx must have shape"):
+        ress.ress_block_sparse_attn(q, q, q, torch.zeros(H + 1, nb, 2, dtype=torch.int32), B)
+    with pytest.raises(ValueError, match="out must have shape"):
+        ress.ress_block_sparse_attn(q, q, q, torch.zeros(H, nb, 2, dtype=torch.int32), B,
+                                    out=torch.zeros(nb * B, H, 32, dtype=bf))
+    with pytest.raises(TypeError, match="lse must be"):
+        ress.ress_block_sparse_attn(q, q, q, torch.zeros(H, nb, 2, dtype=torch.int32), B,
+                                    lse=torch.zeros(H, nb * B, dtype=torch.float64))
+    idx = torch.zeros(H, nb, 2, dtype=torch.int32)
+    lse = torch.zeros(H, nb * B)
+    with pytest.raises(ValueError, match="drift must have shape"):
+        ress.ress_block_drift(q, q, q, idx, lse, B, drift=torch.zeros(H, nb, nb))
+    with pytest.raises(ValueError, match="lse must have shape"):
+        ress.ress_block_drift(q, q, q, idx, torch.zeros(H, nb), B)
+    with pytest.raises(TypeError, match="counts must be"):
+        ress.ress_select_blocks_cdf(q, q, 0.9, B, counts=torch.zeros(H, nb, dtype=torch.int64))
+    with pytest.raises(TypeError, match="workspace must be"):
+        ress.ress_select_blocks(q, q, None, 2, 0.0, B, workspace=torch.zeros(64))
+    with pytest.raises(ValueError, match="idx must have shape"):
+        ress.ress_select_blocks(q, q, None, 2, 0.0, B, idx=torch.zeros(H, nb, 3, dtype=torch.int32))
+    # Consistent host tensors pass every check and stop at the device check.
+    with pytest.raises(ValueError, match="CUDA device"):
+        ress.ress_select_blocks(q, q, None, 2, 0.0, B)
