@@ -55,6 +55,8 @@ MUTATIONS = {
         ("live = valid[rows] & ~special[rows]", "live = valid[rows]"),
     "padding keys in the drift":
         ("toks = toks[valid[toks]]", "toks = toks"),
+    "empty key blocks ranked like the others":
+        ("rank[:, :, empty] = -np.inf", "rank[:, :, empty] = rank[:, :, empty]"),
     "a causal mask over the kept tokens":
         ("s = (q_blk @ keys.T) / math.sqrt(d)\n    m = s.max",
          "s = (q_blk @ keys.T) / math.sqrt(d)\n    s = s + np.triu(np.full(s.shape, -np.inf), 1)\n    m = s.max"),

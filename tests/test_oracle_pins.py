@@ -540,6 +540,40 @@ def test_special_only_key_blocks_are_always_kept():
         assert others == sorted(rest[:1])
 
 
+def test_empty_key_blocks_are_never_preferred_to_non_empty_ones():
+    # Views of 12 tokens with 8 real ones and blocks of 4: block 2 of every
+    # view (positions 8..11) holds only padding and pools to the zero vector,
+    # so its logit is exactly 0.  Every valid key points away from every
+    # query, so every non-empty block has a negative logit: ranked like the
+    # others, the empty blocks would be the top of each row.  The expected
+    # kept set comes from plain means over the valid tokens and a stable
+    # sort of the non-empty blocks alone.
+    rng = np.random.default_rng(17)
+    views, tpv, real, B, H, d = 3, 12, 8, 4, 2, 8
+    n = views * tpv
+    q = np.abs(rng.normal(size=(n, H, d))) + 0.5
+    k = -(np.abs(rng.normal(size=(n, H, d))) + 0.5)
+    valid, special = oracle.view_layout(n, tpv, real, 0)
+    nb, budget = n // B, 4
+    empty = [j for j in range(nb) if not valid[j * B:(j + 1) * B].any()]
+    assert empty == [2, 5, 8]
+    idx = oracle.select_blocks_layout(q, k, B, budget, valid, special)
+    for h in range(H):
+        kbar = {j: k[j * B:(j + 1) * B][valid[j * B:(j + 1) * B], h].mean(axis=0)
+                for j in range(nb) if j not in empty}
+        for i in range(nb):
+            toks = valid[i * B:(i + 1) * B]
+            if not toks.any():
+                continue
+            qbar = q[i * B:(i + 1) * B][toks, h].mean(axis=0)
+            cand = sorted(kbar)
+            s = np.array([qbar @ kbar[j] for j in cand]) / math.sqrt(d)
+            assert (s < 0).all()
+            order = np.argsort(-s, kind="stable")[:budget]
+            assert idx[h, i].tolist() == sorted(cand[o] for o in order)
+            assert not set(empty) & set(idx[h, i].tolist())
+
+
 def test_layout_drift_reconstructs_dense_attention_over_valid_keys():
     q, k, v, valid, special, B = _layout_case(seed=41)
     n, H, d = q.shape
