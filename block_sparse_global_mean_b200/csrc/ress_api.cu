@@ -54,6 +54,34 @@ __global__ void cast_bf16_kernel(const float4* __restrict__ src, uint2* __restri
   }
 }
 
+// One warp per (h, i) row of idx: every entry in [0, nb), strictly ascending.
+__global__ void __launch_bounds__(256) validate_idx_kernel(const int32_t* __restrict__ idx,
+                                                           int rows, int nb, int budget,
+                                                           DeviceError* err) {
+  const int row = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const int32_t* r = idx + (size_t)row * budget;
+  bool out_of_range = false, repeat = false, descending = false;
+  for (int e = lane; e < budget; e += 32) {
+    const int j = r[e];
+    out_of_range |= j < 0 || j >= nb;
+    if (e + 1 < budget) {
+      const int nx = r[e + 1];
+      repeat |= nx == j;
+      descending |= nx < j;
+    }
+  }
+  const unsigned any_range = __ballot_sync(0xffffffffu, out_of_range);
+  const unsigned any_repeat = __ballot_sync(0xffffffffu, repeat);
+  const unsigned any_desc = __ballot_sync(0xffffffffu, descending);
+  if (lane == 0) {
+    if (any_range) raise_device_error(err, RESS_ERR_BAD_INDEX, 80);
+    else if (any_repeat) raise_device_error(err, RESS_ERR_BAD_INDEX, 81);
+    else if (any_desc) raise_device_error(err, RESS_ERR_BAD_INDEX, 82);
+  }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -260,6 +288,22 @@ ress_status ress_block_drift(const ress_shape* shape, const void* q, const void*
     return RESS_ERR_WORKSPACE;
   if ((s = stage_inputs(g, q, k, v, workspace, workspace_bytes, st)) != RESS_OK) return s;
   return launch_drift(g, q, k, v, budget, idx, lse, drift, set_drift, st);
+}
+
+ress_status ress_validate_idx(const ress_shape* shape, int32_t budget, const int32_t* idx,
+                              void* stream) {
+  Geometry g;
+  ress_status s = check_shape(shape, &g);
+  if (s != RESS_OK) return s;
+  if ((s = check_budget(g, budget)) != RESS_OK) return s;
+  if (g.nb == 0) return RESS_OK;
+  if (!idx || (reinterpret_cast<uintptr_t>(idx) & 3u)) return RESS_ERR_INVALID_ARG;
+  DeviceError* err = device_error_ptr();
+  if (err == nullptr) return RESS_ERR_CUDA;
+  const int rows = g.heads * g.nb;
+  validate_idx_kernel<<<(rows + 7) / 8, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      idx, rows, g.nb, budget, err);
+  return record_cuda(cudaGetLastError());
 }
 
 ress_status ress_check_device_errors(void* stream, int32_t* detail) {

@@ -204,7 +204,9 @@ __global__ void __launch_bounds__(kThreads, B128 ? 2 : 1)
       raise_device_error(p.err, RESS_ERR_BAD_INDEX, 2);
       continue;
     }
-    atomicOr(&(s ? keptB : keptA)[j >> 5], 1u << (j & 31));
+    // A block named twice leaves more than nb - budget blocks dropped.
+    if (atomicOr(&(s ? keptB : keptA)[j >> 5], 1u << (j & 31)) & (1u << (j & 31)))
+      raise_device_error(p.err, RESS_ERR_BAD_INDEX, 5);
   }
   __syncthreads();
 

@@ -33,7 +33,7 @@ void* static_scratch_address() {
   std::lock_guard<std::mutex> lock(mu);
   if (cache[dev] == nullptr) {
     void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_select_scratch) != cudaSuccess) return nullptr;
+    if (record_cuda(cudaGetSymbolAddress(&ptr, g_select_scratch)) != RESS_OK) return nullptr;
     cache[dev] = ptr;
   }
   return cache[dev];

@@ -70,6 +70,8 @@ lib.ress_last_cuda_error.restype = ctypes.c_char_p
 lib.ress_last_cuda_error.argtypes = []
 lib.ress_test_exp2.restype = ctypes.c_int
 lib.ress_test_exp2.argtypes = [_P, _P, ctypes.c_int32, _P]
+lib.ress_validate_idx.restype = ctypes.c_int
+lib.ress_validate_idx.argtypes = [_SHAPE, ctypes.c_int32, _P, _P]
 lib.ress_check_device_errors.restype = ctypes.c_int
 lib.ress_check_device_errors.argtypes = [_P, ctypes.POINTER(ctypes.c_int32)]
 
@@ -86,6 +88,13 @@ class RessError(RuntimeError):
 def _check(status: int, where: str) -> None:
     if status != RESS_OK:
         raise RessError(status, where)
+
+
+def _on(device: torch.device, fn, *args) -> int:
+    """Calls ``fn(*args)`` with ``device`` current: the library looks up its
+    per-device state (error flag, fixed scratch) on the current device."""
+    with torch.cuda.device(device):
+        return fn(*args)
 
 
 def make_shape(n: int, heads: int, block: int, dtype: torch.dtype, head_dim: int = 64) -> ress_shape:
@@ -187,7 +196,7 @@ def ress_select_blocks(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tenso
     need = int(lib.ress_select_workspace_bytes(ctypes.byref(sh), ctypes.c_float(lam)))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    status = lib.ress_select_blocks(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(budget),
+    status = _on(q.device, lib.ress_select_blocks, ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(budget),
                                     ctypes.c_float(lam), _ptr(idx), _ptr(workspace),
                                     workspace.numel(), _stream_ptr(stream, q.device))
     _check(status, "ress_select_blocks")
@@ -217,7 +226,7 @@ def ress_select_blocks_cdf(q: torch.Tensor, k: torch.Tensor, tau: float, block: 
     need = int(lib.ress_select_workspace_bytes(ctypes.byref(sh), ctypes.c_float(0.0)))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    status = lib.ress_select_blocks_cdf(ctypes.byref(sh), _ptr(q), _ptr(k), ctypes.c_float(tau),
+    status = _on(q.device, lib.ress_select_blocks_cdf, ctypes.byref(sh), _ptr(q), _ptr(k), ctypes.c_float(tau),
                                         cap, _ptr(counts), _ptr(idx), _ptr(workspace),
                                         workspace.numel(), _stream_ptr(stream, q.device))
     _check(status, "ress_select_blocks_cdf")
@@ -236,7 +245,7 @@ def ress_select_blocks_noalloc(q: torch.Tensor, k: torch.Tensor, v: Optional[tor
     if idx is None:
         idx = torch.empty((h, n // block, budget), dtype=torch.int32, device=q.device)
     _check_buffer(idx, (h, n // block, budget), torch.int32, q.device, "idx")
-    status = lib.ress_select_blocks_noalloc(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(budget),
+    status = _on(q.device, lib.ress_select_blocks_noalloc, ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(budget),
                                             ctypes.c_float(lam), _ptr(idx),
                                             _stream_ptr(stream, q.device))
     _check(status, "ress_select_blocks_noalloc")
@@ -273,7 +282,7 @@ def ress_block_sparse_attn(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, id
     need = int(lib.ress_attn_workspace_bytes(ctypes.byref(sh)))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    status = lib.ress_block_sparse_attn(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(budget),
+    status = _on(q.device, lib.ress_block_sparse_attn, ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(budget),
                                         _ptr(idx), _ptr(out), out_code, _ptr(lse), _ptr(workspace),
                                         0 if workspace is None else workspace.numel(),
                                         _stream_ptr(stream, q.device))
@@ -304,7 +313,7 @@ def ress_block_drift(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: tor
     need = int(lib.ress_attn_workspace_bytes(ctypes.byref(sh)))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
-    status = lib.ress_block_drift(ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(budget),
+    status = _on(q.device, lib.ress_block_drift, ctypes.byref(sh), _ptr(q), _ptr(k), _ptr(v), int(budget),
                                   _ptr(idx), _ptr(lse), _ptr(drift) if drift.numel() else None,
                                   _ptr(set_drift), _ptr(workspace),
                                   0 if workspace is None else workspace.numel(),
@@ -313,10 +322,25 @@ def ress_block_drift(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: tor
     return drift, set_drift
 
 
+def ress_validate_idx(idx: torch.Tensor, n: int, block: int,
+                      stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Checks idx [H, nb, budget] on the device (in range, strictly ascending
+    rows); a bad row shows up in ress_check_device_errors (RESS_ERR_BAD_INDEX,
+    detail 80 out of range, 81 repeated block, 82 not ascending)."""
+    if idx.dim() != 3:
+        raise ValueError(f"idx must be [H, nb, budget], got {tuple(idx.shape)}")
+    h = idx.shape[0]
+    _check_idx(idx, h, n // block, idx.device)
+    sh = make_shape(n, h, block, torch.bfloat16)
+    status = _on(idx.device, lib.ress_validate_idx, ctypes.byref(sh), int(idx.shape[2]), _ptr(idx),
+                 _stream_ptr(stream, idx.device))
+    _check(status, "ress_validate_idx")
+
+
 def ress_check_device_errors(stream: Optional[torch.cuda.Stream] = None,
                              device: Optional[torch.device] = None) -> Tuple[int, int]:
     """Synchronise and return (status, detail) of the device error flag (cleared)."""
     dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
     detail = ctypes.c_int32(0)
-    status = lib.ress_check_device_errors(_stream_ptr(stream, dev), ctypes.byref(detail))
+    status = _on(dev, lib.ress_check_device_errors, _stream_ptr(stream, dev), ctypes.byref(detail))
     return int(status), int(detail.value)

@@ -26,8 +26,10 @@
  * - d must be 64.  The block size B (query blocks and key blocks alike) is 64
  *   or 128, and N must be a multiple of B; nb = N / B.  Padding tokens, if
  *   any, are ordinary tokens to the library.
- * - All data pointers are device pointers owned by the caller.  The library
- *   never allocates, frees or synchronises; every call is asynchronous and
+ * - All data pointers are device pointers owned by the caller, on the
+ *   current device (the library keeps per-device state, such as its error
+ *   flag, and looks it up on the device that is current at the call).
+ *   The library never allocates, frees or synchronises; every call is asynchronous and
  *   ordered on `stream` (a cudaStream_t passed as void*, NULL = the legacy
  *   default stream).  Scratch memory comes from the caller's `workspace`,
  *   sized by the matching *_workspace_bytes() query, 256-byte aligned.
@@ -225,6 +227,9 @@ ress_status ress_block_sparse_attn(const ress_shape* shape, const void* q, const
  *
  *   idx        as for ress_block_sparse_attn, but rows must hold `budget`
  *              distinct in-range blocks (the drift row length is nb - budget).
+ *              A row that names a block twice is flagged (RESS_ERR_BAD_INDEX,
+ *              detail 5, via ress_check_device_errors); the drift entries
+ *              such a row would place beyond nb - budget are not written.
  *   lse        [H][N] float32 from ress_block_sparse_attn.
  *   drift      out, [H][nb][nb - budget] float32 (may be NULL when budget == nb).
  *   set_drift  out, [H][nb] float32, or NULL.
@@ -233,6 +238,22 @@ ress_status ress_block_drift(const ress_shape* shape, const void* q, const void*
                              const void* v, int32_t budget, const int32_t* idx,
                              const float* lse, float* drift, float* set_drift,
                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Debug aid: checks a kept-block list on the device, ordered on `stream`
+ * (VASC A.2: the binary Top-K mask has exact capacity, so a row names
+ * `budget` distinct blocks; ress_select_blocks writes them ascending).
+ * Launches one small kernel that reads idx and writes nothing but the device
+ * error flag: RESS_ERR_BAD_INDEX, reported by ress_check_device_errors with
+ * detail 80 (an entry outside [0, nb)), 81 (a row repeats a block in
+ * adjacent positions) or 82 (a row not in ascending order).  The first error
+ * found wins.
+ *
+ *   idx      [H][nb][budget] int32 device array, 4-byte aligned.
+ *   budget   1 <= budget <= nb.
+ */
+ress_status ress_validate_idx(const ress_shape* shape, int32_t budget, const int32_t* idx,
+                              void* stream);
 
 /*
  * Synchronises `stream`, then reports and clears the device error flag that

@@ -27,6 +27,15 @@ DRIFT_REL = 2e-2
 DRIFT_ABS_FRAC = 1e-4
 
 
+def poison(shape, dtype, device="cuda") -> torch.Tensor:
+    """An output buffer pre-filled with values no kernel writes (NaN for
+    floating point, -1 for integers), so an element the kernel skips cannot
+    pass by holding a plausible earlier result."""
+    if dtype.is_floating_point:
+        return torch.full(shape, float("nan"), dtype=dtype, device=device)
+    return torch.full(shape, -1, dtype=dtype, device=device)
+
+
 def np64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to(torch.float64).cpu().numpy()
 

@@ -8,6 +8,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 from block_sparse_global_mean_b200 import build as ress_build
 
@@ -64,6 +65,13 @@ def _shape(ress, n=512, heads=2, d=64, block=64, dtype=0):
 FAKE = 0x10000          # 16-byte aligned, never dereferenced: every case fails validation
 FAKE_WS = 0x20000       # 256-byte aligned
 
+# The cases below pass placeholder addresses that every host check must reject
+# before a CUDA call.  They run where no GPU is visible, so that even a
+# regressed check could only produce a CUDA error, never a launch on a bad
+# address.
+no_gpu_only = pytest.mark.skipif(torch.cuda.is_available(),
+                                 reason="placeholder-pointer cases run only without a GPU")
+
 
 def _select(ress, shape, q=FAKE, k=FAKE, v=None, budget=4, lam=0.0, idx=FAKE, ws=FAKE_WS,
             ws_bytes=1 << 30):
@@ -71,6 +79,7 @@ def _select(ress, shape, q=FAKE, k=FAKE, v=None, budget=4, lam=0.0, idx=FAKE, ws
                                        budget, ctypes.c_float(lam), idx, ws, ws_bytes, None)
 
 
+@no_gpu_only
 def test_select_rejects_bad_arguments_on_the_host(ress):
     E = ress
     assert _select(ress, None) == E.RESS_ERR_INVALID_ARG
@@ -93,6 +102,7 @@ def test_select_rejects_bad_arguments_on_the_host(ress):
     assert _select(ress, big, budget=1) == E.RESS_ERR_UNSUPPORTED               # nb > 4096
 
 
+@no_gpu_only
 def test_empty_input_is_a_no_op(ress):
     sh = _shape(ress, n=0)
     assert _select(ress, sh, budget=0) == ress.RESS_OK
@@ -102,6 +112,7 @@ def test_empty_input_is_a_no_op(ress):
                                      None, None, 0, None) == ress.RESS_OK
 
 
+@no_gpu_only
 def test_attention_and_drift_reject_bad_arguments_on_the_host(ress):
     sh = _shape(ress)
     lib = ress.lib
@@ -198,3 +209,29 @@ def test_binding_rejects_mismatched_tensors_before_any_library_call(ress):
     # Consistent host tensors pass every check and stop at the device check.
     with pytest.raises(ValueError, match="CUDA device"):
         ress.ress_select_blocks(q, q, None, 2, 0.0, B)
+
+
+@no_gpu_only
+def test_validate_idx_rejects_bad_arguments_on_the_host(ress):
+    sh = _shape(ress)
+    lib = ress.lib
+    assert lib.ress_validate_idx(None, 4, FAKE, None) == ress.RESS_ERR_INVALID_ARG
+    assert lib.ress_validate_idx(ctypes.byref(sh), 0, FAKE, None) == ress.RESS_ERR_INVALID_ARG
+    assert lib.ress_validate_idx(ctypes.byref(sh), 9, FAKE, None) == ress.RESS_ERR_INVALID_ARG
+    assert lib.ress_validate_idx(ctypes.byref(sh), 4, None, None) == ress.RESS_ERR_INVALID_ARG
+    assert lib.ress_validate_idx(ctypes.byref(sh), 4, FAKE + 2, None) == ress.RESS_ERR_INVALID_ARG
+    empty = _shape(ress, n=0)
+    assert lib.ress_validate_idx(ctypes.byref(empty), 0, FAKE, None) == ress.RESS_OK
+
+
+@no_gpu_only
+def test_noalloc_rejects_problems_beyond_its_fixed_scratch(ress):
+    # H = 64, nb = 4,096: about 134 MB of scratch, more than the fixed 32 MiB.
+    big = _shape(ress, n=64 * 4096, heads=64)
+    assert ress.lib.ress_select_blocks_noalloc(ctypes.byref(big), FAKE, FAKE, None, 8,
+                                               ctypes.c_float(0.0), FAKE, None) \
+        == ress.RESS_ERR_WORKSPACE
+    # and argument errors come first, as for the workspace entry point
+    assert ress.lib.ress_select_blocks_noalloc(ctypes.byref(big), FAKE, FAKE, None, 0,
+                                               ctypes.c_float(0.0), FAKE, None) \
+        == ress.RESS_ERR_INVALID_ARG

@@ -1,7 +1,9 @@
 """Stage 2 on the GPU against the oracle (run with the GPU's own idx): every
 row at the small sizes, sampled rows at the full sizes, and the edge cases
 (full budget = dense attention, budget 1, an odd number of query blocks,
-unsorted and duplicated indices, out-of-range indices)."""
+unsorted and duplicated indices, out-of-range indices, one head and the
+64-head maximum, a grid near the 10,000-block limit).  Outputs start
+poisoned (NaN), so an element the kernel skips cannot pass."""
 
 import numpy as np
 import pytest
@@ -9,13 +11,16 @@ import torch
 
 import oracle
 from block_sparse_global_mean_b200 import workloads
-from tests.parity import assert_attn_close, np64, sample_rows
+from tests.parity import assert_attn_close, np64, poison, sample_rows
 
 pytestmark = pytest.mark.gpu
 
 
 def _run(ress, w, q, k, v, idx, out_dtype=None):
-    out, lse = ress.ress_block_sparse_attn(q, k, v, idx, w.block, out_dtype=out_dtype)
+    n, h = q.shape[0], q.shape[1]
+    out = poison(q.shape, out_dtype or q.dtype, q.device)
+    lse = poison((h, n), torch.float32, q.device)
+    out, lse = ress.ress_block_sparse_attn(q, k, v, idx, w.block, out=out, lse=lse)
     status, detail = ress.ress_check_device_errors()
     assert status == 0, (status, detail)
     return out, lse
@@ -127,9 +132,11 @@ def test_out_of_range_indices_are_skipped_and_flagged(ress_gpu):
     idx[0, 1, 2] = 77          # out of range
     idx[0, 3, 0] = -5          # out of range
     out, lse = ress_gpu.ress_block_sparse_attn(q.cuda(), k.cuda(), v.cuda(),
-                                               torch.from_numpy(idx).cuda(), B)
+                                               torch.from_numpy(idx).cuda(), B,
+                                               out=poison((nb * B, H, 64), torch.bfloat16),
+                                               lse=poison((H, nb * B), torch.float32))
     status, detail = ress_gpu.ress_check_device_errors()
-    assert status == ress_gpu.RESS_ERR_BAD_INDEX
+    assert status == ress_gpu.RESS_ERR_BAD_INDEX and detail == 1
     assert ress_gpu.ress_check_device_errors()[0] == 0          # cleared
     qn, kn, vn = np64(q), np64(k), np64(v)
     for i, kept in [(1, [0, 2]), (3, [2, 4]), (0, [0, 2, 4])]:
@@ -144,3 +151,35 @@ def test_float32_inputs_are_staged_and_output_in_float32(ress_gpu, wcache):
     idx = ress_gpu.ress_select_blocks(q, k, None, w.budget, 0.0, w.block)
     out, lse = _run(ress_gpu, w, q, k, v, idx)
     assert out.dtype == torch.float32
+
+
+@pytest.mark.parametrize("heads,nb,budget", [(1, 11, 4), (64, 6, 3)])
+def test_one_head_and_the_64_head_maximum(heads, nb, budget, ress_gpu):
+    B = 64
+    g = torch.Generator().manual_seed(heads + nb)
+    q, k, v = (torch.randn(nb * B, heads, 64, generator=g).to(torch.bfloat16) for _ in range(3))
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    idx = ress_gpu.ress_select_blocks(qd, kd, None, budget, 0.0, B)
+    w = workloads.Workload("heads", 1, nb * B, nb * B, heads, 64, "bf16", B, budget, 0.0, 0, "iid")
+    out, lse = _run(ress_gpu, w, qd, kd, vd, idx, out_dtype=torch.float32)
+    rows = [(h, i) for h in range(heads) for i in range(nb)]
+    _compare_rows(q, k, v, idx.cpu().numpy(), out.cpu(), lse.cpu(), B, rows)
+
+
+def test_grid_near_the_10000_block_limit(ress_gpu):
+    """nb = 9,999 key blocks (the kept-block lists of a tile fill most of the
+    shared memory): one head, budget 3, sampled rows including the last
+    (half-empty) tile."""
+    H, nb, B, budget = 1, 9999, 64, 3
+    g = torch.Generator().manual_seed(99)
+    q, k, v = (torch.randn(nb * B, H, 64, generator=g).to(torch.bfloat16) for _ in range(3))
+    rng = np.random.default_rng(99)
+    idx = np.sort(np.stack([rng.choice(nb, budget, replace=False) for _ in range(nb)]), -1)
+    idx[0] = [0, nb // 2, nb - 1]
+    idx = idx.astype(np.int32)[None]
+    w = workloads.Workload("wide", 1, nb * B, nb * B, H, 64, "bf16", B, budget, 0.0, 0, "iid")
+    out, lse = _run(ress_gpu, w, q.cuda(), k.cuda(), v.cuda(), torch.from_numpy(idx).cuda(),
+                    out_dtype=torch.float32)
+    rows = [(0, i) for i in (0, 1, 2, 5000, 7777, nb - 2, nb - 1)]
+    _compare_rows(q, k, v, idx, out.cpu(), lse.cpu(), B, rows)
+    assert torch.isfinite(out).all()

@@ -8,13 +8,22 @@ import torch
 
 import oracle
 from block_sparse_global_mean_b200 import workloads
-from tests.parity import MASK_MARGIN, assert_attn_close, np64
+from tests.parity import MASK_MARGIN, assert_attn_close, np64, poison
 
 pytestmark = pytest.mark.gpu
 
 # The count may differ from float64 only where the cumulative mass is this
 # close to tau (float32 probabilities; the GPU's running sum itself is exact).
 CDF_MASS_EPS = 1e-5
+
+
+def _cdf(ress, q, k, tau, block, capacity=None):
+    """ress_select_blocks_cdf with poisoned (-1) counts and idx buffers."""
+    h, nb = q.shape[1], q.shape[0] // block
+    cap = nb if capacity is None else capacity
+    return ress.ress_select_blocks_cdf(q, k, tau, block, capacity=capacity,
+                                       counts=poison((h, nb), torch.int32, q.device),
+                                       idx=poison((h, nb, cap), torch.int32, q.device))
 
 
 def _check_errors(ress):
@@ -66,12 +75,12 @@ def test_cdf_selection_matches_oracle(name, tau, ress_gpu, wcache):
     w = workloads.WORKLOADS[name]
     q, k, _ = wcache.get(w)
     tau = float(np.float32(tau))
-    counts, idx = ress_gpu.ress_select_blocks_cdf(q, k, tau, w.block)
+    counts, idx = _cdf(ress_gpu, q, k, tau, w.block)
     _check_errors(ress_gpu)
     sc = oracle.selection_scores(np64(q), np64(k), None, w.block, 0.0)
     _assert_cdf_parity(counts.cpu().numpy(), idx.cpu().numpy(), sc["probs"], sc["logits"], tau,
                        w.n_blocks)
-    again_c, again_i = ress_gpu.ress_select_blocks_cdf(q, k, tau, w.block)
+    again_c, again_i = _cdf(ress_gpu, q, k, tau, w.block)
     assert torch.equal(again_c, counts) and torch.equal(again_i, idx)     # deterministic
 
 
@@ -83,7 +92,7 @@ def test_cdf_constant_rows_keep_the_lowest_indices(ress_gpu):
     q = torch.zeros(nb * B, H, 64)
     k = torch.randn(nb * B, H, 64, generator=g)
     tau = float(np.float32(0.4567))
-    counts, idx = ress_gpu.ress_select_blocks_cdf(q.cuda(), k.cuda(), tau, B, capacity=200)
+    counts, idx = _cdf(ress_gpu, q.cuda(), k.cuda(), tau, B, capacity=200)
     _check_errors(ress_gpu)
     want = int(np.ceil(tau * nb))
     assert (counts.cpu() == want).all()
@@ -109,7 +118,7 @@ def test_cdf_crowded_bin_of_distinct_logits(ress_gpu):
     sc = oracle.selection_scores(np64(q), np64(k), None, B, 0.0)
     for tau in (0.3, 0.7, 0.95):
         tau = float(np.float32(tau))
-        counts, idx = ress_gpu.ress_select_blocks_cdf(q.cuda(), k.cuda(), tau, B)
+        counts, idx = _cdf(ress_gpu, q.cuda(), k.cuda(), tau, B)
         _check_errors(ress_gpu)
         _assert_cdf_parity(counts.cpu().numpy(), idx.cpu().numpy(), sc["probs"], sc["logits"],
                            tau, nb)
@@ -119,7 +128,7 @@ def test_cdf_truncates_to_the_capacity_and_feeds_attention(ress_gpu, wcache):
     w = workloads.WORKLOADS["vggt8"]
     q, k, v = wcache.get(w)
     tau, cap = float(np.float32(0.95)), 40
-    counts, idx = ress_gpu.ress_select_blocks_cdf(q, k, tau, w.block, capacity=cap)
+    counts, idx = _cdf(ress_gpu, q, k, tau, w.block, capacity=cap)
     _check_errors(ress_gpu)
     sc = oracle.selection_scores(np64(q), np64(k), None, w.block, 0.0)
     _assert_cdf_parity(counts.cpu().numpy(), idx.cpu().numpy(), sc["probs"], sc["logits"], tau, cap)

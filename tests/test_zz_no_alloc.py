@@ -5,7 +5,8 @@ in a row (the fixed scratch array keeps the previous call's contents).
 Some callers cannot allocate device memory (a plugin inside another
 framework's allocator, or a loop where an allocation is not allowed); they
 use ress_select_blocks_noalloc.  This file is collected last so that a run
-that stops at the first failure has already run every other test."""
+that stops at the first failure has already run every other test.  The
+oversized-problem rejection, which needs no GPU, is in test_abi_cpu.py."""
 
 import ctypes
 
@@ -13,6 +14,7 @@ import pytest
 import torch
 
 from block_sparse_global_mean_b200 import workloads
+from tests.parity import poison
 
 pytestmark = pytest.mark.gpu
 
@@ -26,12 +28,18 @@ def _call_noalloc(ress, w, q, k, v, idx):
     return status
 
 
-@pytest.mark.parametrize("name", ["vggt8", "views32"])
+def _reference(ress, w, q, k, v):
+    ref = ress.ress_select_blocks(q, k, v if w.lam else None, w.budget, w.lam, w.block,
+                                  idx=poison((w.heads, w.n_blocks, w.budget), torch.int32))
+    assert ress.ress_check_device_errors()[0] == 0
+    return ref
+
+
+@pytest.mark.parametrize("name", ["tiny", "vggt8", "views32"])
 def test_noalloc_matches_workspace_entry_point_on_two_calls(name, ress_gpu):
     w = workloads.WORKLOADS[name]
     q, k, v = workloads.generate(w, device="cuda")
-    ref = ress_gpu.ress_select_blocks(q, k, v if w.lam else None, w.budget, w.lam, w.block)
-    assert ress_gpu.ress_check_device_errors()[0] == 0
+    ref = _reference(ress_gpu, w, q, k, v)
     for _ in range(2):
         idx = torch.full_like(ref, -1)
         assert _call_noalloc(ress_gpu, w, q, k, v, idx) == ress_gpu.RESS_OK
@@ -40,11 +48,15 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(name, ress_gpu):
         assert torch.equal(idx, ref)
 
 
-def test_noalloc_rejects_problems_beyond_its_fixed_scratch(ress_gpu):
-    # H = 64, nb = 4,096: about 134 MB of scratch, more than the fixed 32 MiB.
-    w = workloads.Workload("big", 1, 64 * 4096, 64 * 4096, 64, 64, "bf16", 64, 8, 0.0, 0, "iid")
-    sh = ress_gpu.make_shape(w.n_tokens, w.heads, w.block, torch.bfloat16)
-    fake = 1 << 20     # aligned, never dereferenced: the call returns before any launch
-    status = ress_gpu.lib.ress_select_blocks_noalloc(ctypes.byref(sh), fake, fake, None, 8,
-                                                     ctypes.c_float(0.0), fake, None)
-    assert status == ress_gpu.RESS_ERR_WORKSPACE
+def test_a_smaller_call_after_a_larger_one(ress_gpu):
+    """Calls of different sizes share the array: the 32-view call with the
+    value contrast fills more of it than the 8-view call that follows, which
+    must read only what it wrote itself."""
+    for name in ["views32", "vggt8", "tiny", "views32"]:
+        w = workloads.WORKLOADS[name]
+        q, k, v = workloads.generate(w, device="cuda")
+        ref = _reference(ress_gpu, w, q, k, v)
+        idx = torch.full_like(ref, -1)
+        assert _call_noalloc(ress_gpu, w, q, k, v, idx) == ress_gpu.RESS_OK
+        assert ress_gpu.ress_check_device_errors()[0] == 0
+        assert torch.equal(idx, ref), name
