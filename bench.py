@@ -10,7 +10,9 @@ H = 16, d = 64, block 64, 220 of 2,200 key blocks kept (90 % sparsity).
 
 With N > 1 launch one process per GPU with torch.distributed.run; every rank
 processes its own input (weak scaling, no data-path collective) and rank 0
-prints one JSON line.  `--impl reference` times the CPU oracle instead (rank 0
+prints one JSON line.  With --shard heads the ranks split the heads of one
+input instead (strong scaling; every stage is independent per head, so there
+is still no data-path collective).  `--impl reference` times the CPU oracle instead (rank 0
 only), on bounded samples of the same workload.
 """
 
@@ -155,12 +157,33 @@ def parse_args():
     ap.add_argument("--no-dense", action="store_true", help="skip the dense SDPA comparison")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU oracle baseline")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the 200-view record (selection, attention and drift stages)")
+    ap.add_argument("--shard", default="none", choices=["none", "heads"],
+                    help="none: every rank runs its own input (weak scaling); heads: the ranks "
+                         "split the heads of one input (strong scaling, no collective)")
     return ap.parse_args()
 
 
 def rank_seed(w, rank: int) -> int:
     """Every rank draws its own input (weak scaling over independent inputs)."""
     return w.seed + 1000 * rank
+
+
+def head_slice(heads: int, world: int, rank: int):
+    """Heads [h0, h1) of rank `rank` when `world` ranks split one input by head
+    (every stage is independent per head: no exchange step)."""
+    if heads % world != 0:
+        raise ValueError(f"{heads} heads do not split evenly over {world} ranks")
+    per = heads // world
+    return rank * per, (rank + 1) * per
+
+
+def shard_heads(tensors, h0: int, h1: int):
+    """The rank-local, contiguous [N, h1 - h0, d] copies of [N, H, d] tensors:
+    what a rank holds when the projections that produce Q, K, V are split by
+    head."""
+    return tuple(t[:, h0:h1].contiguous() for t in tensors)
 
 
 def max_over_ranks(values, device, world: int):
@@ -177,16 +200,20 @@ def whole_job_tflops(flops_per_step: float, steps: int, world: int, max_elapsed_
     return flops_per_step * steps * world / (max_elapsed_ms / 1e3) / 1e12
 
 
-def workload_config(w, world: int):
+def workload_config(w, world: int, shard: str = "none"):
+    if shard == "heads":
+        par = f"heads/{world} (one input; rank r computes heads [r*H/{world}, (r+1)*H/{world}))"
+    else:
+        par = f"dp{world} (independent inputs per rank)"
     return {
         "workload": (f"{w.name}: {w.views} views x {w.tokens_per_view} tokens (N={w.n_tokens}), "
                      f"H={w.heads}, d={w.head_dim}, block {w.block}, budget {w.budget} of "
                      f"{w.n_blocks} ({100 * w.sparsity:.0f}% sparsity), lambda {w.lam}"),
-        "global_batch": world,
+        "global_batch": 1 if shard == "heads" else world,
         "tokens_per_rank": w.n_tokens,
         "step": "select(pool+score+topk) -> block-sparse attention" + (" -> drift" if w.drift else ""),
         "l2": l2_policy(w)[1],
-        "parallelism": f"dp{world} (independent inputs per rank)",
+        "parallelism": par,
     }
 
 
@@ -194,17 +221,20 @@ def workload_config(w, world: int):
 # CPU oracle timing (the reported baseline)
 # --------------------------------------------------------------------------
 
-def cpu_oracle_rate(w, q_cpu, k_cpu, v_cpu, seconds_target: float = 12.0):
+def cpu_oracle_rate(w, q_cpu, k_cpu, v_cpu, seconds_target: float = 12.0, threads=None):
     """Times the CPU oracle on a bounded sample of one step and extrapolates to
-    the full step.  Returns (TFLOPS, sample description, threads)."""
+    the full step.  `threads` limits the BLAS pool behind the oracle's matmuls
+    (None: as configured, all cores by default).  Returns (TFLOPS, sample
+    description, threads used)."""
+    from threadpoolctl import threadpool_info, threadpool_limits
+
+    if threads is not None:
+        with threadpool_limits(limits=threads):
+            return cpu_oracle_rate(w, q_cpu, k_cpu, v_cpu, seconds_target, None)
     import numpy as np
 
     import oracle
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
-    except Exception:  # noqa: BLE001
-        threads = os.cpu_count() or 1
+    threads = max([d.get("num_threads", 1) for d in threadpool_info()] + [1])
     h0 = 0
     qh = q_cpu[:, h0:h0 + 1].double().numpy()
     kh = k_cpu[:, h0:h0 + 1].double().numpy()
@@ -265,6 +295,161 @@ def run_reference(args, rank: int, world: int):
 # Our arm
 # --------------------------------------------------------------------------
 
+class StepRunner:
+    """One step of the hot path (selection -> attention [-> drift]) on fixed
+    device buffers, with optional CUDA events per stage."""
+
+    def __init__(self, ress, w, heads: int, dev, stream, out_buffers: int = 1):
+        self.ress, self.w, self.stream = ress, w, stream
+        nb, B = w.n_blocks, w.block
+        self.idx = torch.empty((heads, nb, w.budget), dtype=torch.int32, device=dev)
+        self.outs = [torch.empty((w.n_tokens, heads, w.head_dim), dtype=torch.bfloat16, device=dev)
+                     for _ in range(out_buffers)]
+        self.lse = torch.empty((heads, w.n_tokens), dtype=torch.float32, device=dev)
+        self.ws = torch.empty(max(1, ress.select_workspace_bytes(w.n_tokens, heads, B,
+                                                                 torch.bfloat16, w.lam)),
+                              dtype=torch.uint8, device=dev)
+        self.drift = self.set_drift = None
+        if w.drift:
+            self.drift = torch.empty((heads, nb, nb - w.budget), dtype=torch.float32, device=dev)
+            self.set_drift = torch.empty((heads, nb), dtype=torch.float32, device=dev)
+        self.ev = {n: [] for n in ("sel0", "sel1", "att0", "att1", "dr0", "dr1")}
+        self.launches_per_step = (3 if w.lam else 2) + 1 + (1 if w.drift else 0)
+
+    def _mark(self, name, record):
+        if record:
+            e = torch.cuda.Event(enable_timing=True)
+            e.record(self.stream)
+            self.ev[name].append(e)
+
+    def step(self, q, k, v, record=False, out_slot=0):
+        w, r, st = self.w, self.ress, self.stream
+        out = self.outs[out_slot]
+        self._mark("sel0", record)
+        r.ress_select_blocks(q, k, v if w.lam else None, w.budget, w.lam, w.block, idx=self.idx,
+                             workspace=self.ws, stream=st)
+        self._mark("sel1", record)
+        self._mark("att0", record)
+        r.ress_block_sparse_attn(q, k, v, self.idx, w.block, out=out, lse=self.lse, stream=st)
+        self._mark("att1", record)
+        if w.drift:
+            self._mark("dr0", record)
+            r.ress_block_drift(q, k, v, self.idx, self.lse, w.block, drift=self.drift,
+                               set_drift=self.set_drift, stream=st)
+            self._mark("dr1", record)
+        return out
+
+    def mean_ms(self, a, b):
+        ev = self.ev
+        return sum(x.elapsed_time(y) for x, y in zip(ev[a], ev[b])) / max(1, len(ev[a]))
+
+
+def e2e_overlapped(runner, hosts, out_h, steps: int, warmup: int, dev, barrier):
+    """The same step through the public API with host buffers, pipelined over
+    three streams: the H2D copies of step i+1 (pinned memory, one
+    cudaMemcpyAsync per tensor) and the D2H copy of step i-1 run on copy
+    streams while step i computes.  Inputs and outputs are double-buffered.
+    Returns the device time from the first copy of the first timed step to
+    the end of the last copy back (ms)."""
+    comp = runner.stream
+    h2d = torch.cuda.Stream(dev)
+    d2h = torch.cuda.Stream(dev)
+    bufs = [tuple(torch.empty(t.shape, dtype=t.dtype, device=dev) for t in hosts) for _ in range(2)]
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    in_free = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    out_free = [torch.cuda.Event() for _ in range(2)]
+
+    def run(n, timed):
+        e0 = e1 = None
+        for i in range(n):
+            s = i % 2
+            if i >= 2:
+                h2d.wait_event(in_free[s])
+            if timed and i == 0:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e0.record(h2d)
+            with torch.cuda.stream(h2d):
+                for dst, src in zip(bufs[s], hosts):
+                    dst.copy_(src, non_blocking=True)
+            in_ready[s].record(h2d)
+            comp.wait_event(in_ready[s])
+            if i >= 2:
+                comp.wait_event(out_free[s])
+            runner.step(*bufs[s], out_slot=s)
+            in_free[s].record(comp)
+            done[s].record(comp)
+            d2h.wait_event(done[s])
+            with torch.cuda.stream(d2h):
+                out_h[s].copy_(runner.outs[s], non_blocking=True)
+            out_free[s].record(d2h)
+        if timed:
+            e1 = torch.cuda.Event(enable_timing=True)
+            e1.record(d2h)
+        torch.cuda.synchronize(dev)
+        return e0, e1
+
+    run(max(2, warmup), False)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0, e1 = run(steps, True)
+    barrier()
+    return e0.elapsed_time(e1)
+
+
+def union_inflation(idx, block: int) -> float:
+    """Tensor work the attention kernel issues per unit of effective work.
+
+    With 64-token blocks a 128-row tile pairs query blocks 2t and 2t+1 and
+    walks the union of their kept sets, two key blocks per 128-key chunk; it
+    issues ceil(|union| / 2) chunks where the two rows need 2 * budget / 2 =
+    budget chunk-equivalents.  With 128-token blocks the ratio is 1."""
+    import numpy as np
+
+    if block != 64:
+        return 1.0
+    a = idx.cpu().numpy()
+    h, nb, budget = a.shape
+    pairs = nb // 2
+    m = np.zeros((h, pairs, nb), dtype=bool)
+    hh = np.arange(h)[:, None, None]
+    tt = np.arange(pairs)[None, :, None]
+    m[hh, tt, a[:, 0:2 * pairs:2]] = True
+    m[hh, tt, a[:, 1:2 * pairs:2]] = True
+    union = m.sum(-1)
+    chunks = (union + 1) // 2
+    return float(chunks.sum() * 2.0 / (h * pairs * budget))
+
+
+def stage_record(ress, w, dev, steps: int = 3, warmup: int = 1):
+    """CUDA-event times of each stage of `w` over a few steps (rank 0, N = 1):
+    the record of the drift stage, which the 100-view step does not run."""
+    q, k, v = workloads.generate(w, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    runner = StepRunner(ress, w, w.heads, dev, stream)
+    for _ in range(warmup):
+        runner.step(q, k, v)
+    torch.cuda.synchronize(dev)
+    for _ in range(steps):
+        runner.step(q, k, v, record=True)
+    torch.cuda.synchronize(dev)
+    status, detail = ress.ress_check_device_errors(stream, dev)
+    if status != 0:
+        raise RuntimeError(f"device error {status} (detail {detail}) in the {w.name} record")
+    sel, att = runner.mean_ms("sel0", "sel1"), runner.mean_ms("att0", "att1")
+    rec = {"workload": f"{w.name}: N={w.n_tokens}, H={w.heads}, block {w.block}, budget "
+                       f"{w.budget} of {w.n_blocks}", "steps": steps,
+           "select_ms": sel, "attn_ms": att,
+           "attn_tflops": w.effective_flops() / (att / 1e3) / 1e12}
+    if w.drift:
+        dr = runner.mean_ms("dr0", "dr1")
+        rec["drift_ms"] = dr
+        rec["drift_tflops"] = w.drift_flops() / (dr / 1e3) / 1e12
+    del q, k, v, runner
+    torch.cuda.empty_cache()
+    return rec
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch.distributed as dist
 
@@ -274,49 +459,26 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     dev = torch.device("cuda", local_rank)
     w = workloads.WORKLOADS[args.workload]
     peaks, peak_kind = load_peaks()
-    q_cpu, k_cpu, v_cpu = workloads.generate(w, seed=rank_seed(w, rank))
+    if args.shard == "heads":
+        h0, h1 = head_slice(w.heads, world, rank)
+        full = workloads.generate(w)            # the same input on every rank
+        q_cpu, k_cpu, v_cpu = shard_heads(full, h0, h1)
+        del full
+    else:
+        h0, h1 = 0, w.heads
+        q_cpu, k_cpu, v_cpu = workloads.generate(w, seed=rank_seed(w, rank))
+    H = h1 - h0
     q, k, v = (t.to(dev) for t in (q_cpu, k_cpu, v_cpu))
     stream = torch.cuda.current_stream(dev)
-    nb, H, B = w.n_blocks, w.heads, w.block
-    lam = w.lam
-    idx = torch.empty((H, nb, w.budget), dtype=torch.int32, device=dev)
-    out = torch.empty_like(q)
-    lse = torch.empty((H, w.n_tokens), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(1, ress.select_workspace_bytes(w.n_tokens, H, B, q.dtype, lam)),
-                     dtype=torch.uint8, device=dev)
-    drift = set_drift = None
-    if w.drift:
-        drift = torch.empty((H, nb, nb - w.budget), dtype=torch.float32, device=dev)
-        set_drift = torch.empty((H, nb), dtype=torch.float32, device=dev)
-    launches_per_step = (3 if lam else 2) + 1 + (1 if w.drift else 0)
-
-    ev = {n: [] for n in ("sel0", "sel1", "att0", "att1", "dr0", "dr1")}
-
-    def step(qq, kk, vv, record=False):
-        if record:
-            e = torch.cuda.Event(enable_timing=True); e.record(stream); ev["sel0"].append(e)
-        ress.ress_select_blocks(qq, kk, vv if lam else None, w.budget, lam, B, idx=idx, workspace=ws,
-                                stream=stream)
-        if record:
-            e = torch.cuda.Event(enable_timing=True); e.record(stream); ev["sel1"].append(e)
-            e = torch.cuda.Event(enable_timing=True); e.record(stream); ev["att0"].append(e)
-        ress.ress_block_sparse_attn(qq, kk, vv, idx, B, out=out, lse=lse, stream=stream)
-        if record:
-            e = torch.cuda.Event(enable_timing=True); e.record(stream); ev["att1"].append(e)
-        if w.drift:
-            if record:
-                e = torch.cuda.Event(enable_timing=True); e.record(stream); ev["dr0"].append(e)
-            ress.ress_block_drift(qq, kk, vv, idx, lse, B, drift=drift, set_drift=set_drift,
-                                  stream=stream)
-            if record:
-                e = torch.cuda.Event(enable_timing=True); e.record(stream); ev["dr1"].append(e)
+    runner = StepRunner(ress, w, H, dev, stream, out_buffers=2)
+    nb = w.n_blocks
 
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local_rank])
 
     for _ in range(args.warmup):
-        step(q, k, v)
+        runner.step(q, k, v)
     torch.cuda.synchronize(dev)
     status, detail = ress.ress_check_device_errors(stream, dev)
     if status != 0:
@@ -335,54 +497,31 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     for it in range(args.steps):
         if flush:
             scratch.fill_(it & 255)
-        step(q, k, v, record=True)
+        runner.step(q, k, v, record=True)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier()
     if flush:
         # Each step from its first to its last event; the flushes lie between.
-        last = ev["dr1"] if w.drift else ev["att1"]
-        elapsed_ms = sum(a.elapsed_time(b) for a, b in zip(ev["sel0"], last))
+        last = runner.ev["dr1"] if w.drift else runner.ev["att1"]
+        elapsed_ms = sum(a.elapsed_time(b) for a, b in zip(runner.ev["sel0"], last))
     else:
         elapsed_ms = t_start.elapsed_time(t_end)
 
-    def mean_pair(a, b):
-        return sum(x.elapsed_time(y) for x, y in zip(ev[a], ev[b])) / max(1, len(ev[a]))
-
-    sel_ms = mean_pair("sel0", "sel1")
-    att_ms = mean_pair("att0", "att1")
-    dr_ms = mean_pair("dr0", "dr1") if w.drift else None
+    sel_ms = runner.mean_ms("sel0", "sel1")
+    att_ms = runner.mean_ms("att0", "att1")
+    dr_ms = runner.mean_ms("dr0", "dr1") if w.drift else None
 
     # End to end through the public API with host buffers: H2D of Q, K, V from
-    # pinned memory, the step, D2H of the output.
+    # pinned memory, the step, D2H of the output, pipelined across steps.
     e2e = None
     if not args.no_e2e:
-        qh, kh, vh = (t.pin_memory() for t in (q_cpu, k_cpu, v_cpu))
-        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-
-        def e2e_step():
-            qd.copy_(qh, non_blocking=True)
-            kd.copy_(kh, non_blocking=True)
-            vd.copy_(vh, non_blocking=True)
-            step(qd, kd, vd)
-            out_h.copy_(out, non_blocking=True)
-
-        for _ in range(max(1, args.warmup // 2)):
-            e2e_step()
-        barrier()
-        torch.cuda.synchronize(dev)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        e2e_ms = e0.elapsed_time(e1)
-        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
-        d2h = out_h.numel() * out_h.element_size()
+        hosts = tuple(t.pin_memory() for t in (q_cpu, k_cpu, v_cpu))
+        out_h = [torch.empty(runner.outs[0].shape, dtype=runner.outs[0].dtype).pin_memory()
+                 for _ in range(2)]
+        e2e_ms = e2e_overlapped(runner, hosts, out_h, args.steps, args.warmup, dev, barrier)
+        h2d = sum(t.numel() * t.element_size() for t in hosts)
+        d2h = out_h[0].numel() * out_h[0].element_size()
         e2e = {"ms": e2e_ms, "h2d": h2d, "d2h": d2h}
     clock_info = clocks.stop()
 
@@ -397,15 +536,26 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if not args.no_dense and rank == 0:
         dense = dense_baseline(q, k, v, stream)
 
+    extra = None
+    if rank == 0 and world == 1 and not args.no_extra and w.name == "views100":
+        del q, k, v
+        torch.cuda.empty_cache()
+        extra = {"views200": stage_record(ress, workloads.WORKLOADS["views200"], dev)}
+
     if rank != 0:
         return
-    flops = w.effective_flops()
-    value = whole_job_tflops(flops, args.steps, world, elapsed_ms)
-    att_tflops = flops / (att_ms / 1e3) / 1e12
+    flops_rank = w.effective_flops() * H / w.heads
+    if args.shard == "heads":
+        value = w.effective_flops() * args.steps / (elapsed_ms / 1e3) / 1e12
+        e2e_value = w.effective_flops() * args.steps / (e2e_ms / 1e3) / 1e12 if e2e else None
+    else:
+        value = whole_job_tflops(flops_rank, args.steps, world, elapsed_ms)
+        e2e_value = whole_job_tflops(flops_rank, args.steps, world, e2e_ms) if e2e else None
+    att_tflops = flops_rank / (att_ms / 1e3) / 1e12
     peak_tf = float(peaks["bf16_tflops"])
     peak_tf_sus = float(peaks.get("bf16_tflops_sustained", peak_tf))
     sel_bytes = 2 * w.n_tokens * H * 64 * 2 + H * nb * w.budget * 4
-    if lam:
+    if w.lam:
         sel_bytes += w.n_tokens * H * 64 * 2
     sel_gbs = sel_bytes / (sel_ms / 1e3) / 1e9
     line = {
@@ -417,11 +567,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "warmup": args.warmup,
         "ms_per_step": elapsed_ms / args.steps,
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong" if args.shard == "heads" else "weak",
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded clustered multi-view tokens; no dataset or weights)",
-        "config": workload_config(w, world),
+        "config": workload_config(w, world, args.shard),
         "roofline": {
             "kernel": "block_sparse_attn_kernel",
             "bound": "tensor",
@@ -431,8 +581,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "frac": att_tflops / peak_tf,
             "peak_kind": f"{peak_kind} bf16 burst",
             "frac_of_sustained": att_tflops / peak_tf_sus,
-            "traffic": recorded_traffic(w.name),
-            "algorithmic": "4*N*kept_keys*d*H = %.4g FLOP per launch" % flops,
+            "traffic": recorded_traffic(w.name) if H == w.heads else None,
+            "algorithmic": "4*N*kept_keys*d*H = %.4g FLOP per launch" % flops_rank,
         },
         "stages": {
             "select_ms": sel_ms,
@@ -441,25 +591,33 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             "select_bytes": sel_bytes,
             "attn_ms": att_ms,
             "attn_tflops": att_tflops,
+            "attn_union_inflation": union_inflation(runner.idx, w.block),
         },
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": runner.launches_per_step * args.steps,
         "clocks": clock_info,
     }
     if w.drift:
         line["stages"]["drift_ms"] = dr_ms
-        line["stages"]["drift_tflops"] = w.drift_flops() / (dr_ms / 1e3) / 1e12
+        line["stages"]["drift_tflops"] = w.drift_flops() * H / w.heads / (dr_ms / 1e3) / 1e12
     if dense:
         line["dense"] = dense
         line["dense"]["speedup_vs_sparse_attn"] = dense["ms"] / att_ms
         line["dense"]["speedup_vs_step"] = dense["ms"] / (elapsed_ms / args.steps)
     if e2e:
-        line["e2e"] = {"value": whole_job_tflops(flops, args.steps, world, e2e_ms), "unit": "TFLOPS",
+        line["e2e"] = {"value": e2e_value, "unit": "TFLOPS",
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                       "ms_per_step": e2e_ms / args.steps}
+                       "ms_per_step": e2e_ms / args.steps,
+                       "pipelining": "H2D of step i+1 and D2H of step i-1 overlap step i "
+                                     "(two copy streams, double-buffered inputs and outputs)"}
+    if extra:
+        line["extra"] = extra
     if world == 1 and not args.no_cpu:
         rate, sample, threads = cpu_oracle_rate(w, q_cpu, k_cpu, v_cpu)
+        rate1, sample1, _ = cpu_oracle_rate(w, q_cpu, k_cpu, v_cpu, threads=1)
         line["cpu_baseline"] = {"value": rate, "unit": "TFLOPS", "cores": threads,
-                                "kind": "oracle", "sample": sample}
+                                "kind": "oracle", "sample": sample,
+                                "single_thread": {"value": rate1, "unit": "TFLOPS", "cores": 1,
+                                                  "sample": sample1}}
     print(json.dumps(line), flush=True)
 
 

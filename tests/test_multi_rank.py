@@ -1,6 +1,8 @@
 """Host-side logic of the multi-GPU run on the CPU with the gloo backend and
 two ranks: every rank draws its own input, timings are reduced as the maximum
-over ranks, and the whole-job value counts the units of all ranks."""
+over ranks, and the whole-job value counts the units of all ranks; with the
+head split, each rank computes its heads of one input (the oracle stands in
+for the kernels) and the gathered result equals the unsharded one."""
 
 import os
 import socket
@@ -72,3 +74,62 @@ def test_reference_arm_exits_quietly_on_other_ranks():
                        timeout=300)
     assert r.returncode == 0
     assert r.stdout.strip() == ""
+
+
+def _head_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import numpy as np
+
+    import bench
+    import oracle
+    from block_sparse_global_mean_b200 import workloads
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = workloads.scaled(workloads.WORKLOADS["vggt8"], 1, name="split")   # 1,408 tokens, H=16
+        full = workloads.generate(w)
+        h0, h1 = bench.head_slice(w.heads, world, rank)
+        qs, ks, vs = (t.double().numpy() for t in bench.shard_heads(full, h0, h1))
+        assert qs.flags["C_CONTIGUOUS"] and qs.shape[1] == h1 - h0
+        idx = oracle.select_blocks(qs, ks, None, w.block, w.budget)
+        rows = [(h, i) for h in range(h1 - h0) for i in (0, w.n_blocks - 1)]
+        out, lse = oracle.sparse_attention(qs, ks, vs, idx, w.block, rows=rows)
+        parts = [None] * world
+        dist.all_gather_object(parts, (h0, h1, idx, out, lse))
+        if rank == 0:
+            qf, kf, vf = (t.double().numpy() for t in full)
+            ref_idx = oracle.select_blocks(qf, kf, None, w.block, w.budget)
+            ok = True
+            for a, b, idx_r, out_r, lse_r in parts:
+                ok &= np.array_equal(idx_r, ref_idx[a:b])
+                rows_f = [(a + h, i) for h in range(b - a) for i in (0, w.n_blocks - 1)]
+                ref_o, ref_l = oracle.sparse_attention(qf, kf, vf, ref_idx, w.block, rows=rows_f)
+                ok &= np.allclose(out_r, ref_o[:, a:b], equal_nan=True, atol=1e-12)
+                ok &= np.allclose(lse_r, ref_l[a:b], equal_nan=True, atol=1e-12)
+            covered = sorted(h for a, b, *_ in parts for h in range(a, b))
+            q.put((ok, covered))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_head_split_over_two_gloo_ranks_equals_the_unsharded_result():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_head_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    ok, covered = q.get(timeout=300)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert ok
+    assert covered == list(range(16))
+
+
+def test_head_slice_rejects_uneven_splits():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.head_slice(16, 4, 3) == (12, 16)
+    with pytest.raises(ValueError):
+        bench.head_slice(16, 3, 0)
