@@ -536,6 +536,27 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if not args.no_dense and rank == 0:
         dense = dense_baseline(q, k, v, stream)
 
+    # The CDF-threshold selection (SparseVGGT's rule) on the same input, for
+    # its cost relative to the fixed budget: tau = 0.9, capacity = budget.
+    cdf_ms = None
+    if rank == 0 and not args.no_extra:
+        counts = torch.empty((H, nb), dtype=torch.int32, device=dev)
+        cidx = torch.empty((H, nb, w.budget), dtype=torch.int32, device=dev)
+        ws_cdf = torch.empty(max(1, ress.select_workspace_bytes(w.n_tokens, H, w.block, q.dtype, 0.0)),
+                             dtype=torch.uint8, device=dev)
+        ress.ress_select_blocks_cdf(q, k, 0.9, w.block, capacity=w.budget, counts=counts, idx=cidx,
+                                    workspace=ws_cdf, stream=stream)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(5):
+            ress.ress_select_blocks_cdf(q, k, 0.9, w.block, capacity=w.budget, counts=counts,
+                                        idx=cidx, workspace=ws_cdf, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        cdf_ms = e0.elapsed_time(e1) / 5
+        del counts, cidx, ws_cdf
+
     extra = None
     if rank == 0 and world == 1 and not args.no_extra and w.name == "views100":
         del q, k, v
@@ -596,6 +617,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         "gpu_launches": runner.launches_per_step * args.steps,
         "clocks": clock_info,
     }
+    if cdf_ms is not None:
+        line["stages"]["select_cdf_ms"] = cdf_ms
+        line["stages"]["select_cdf"] = "CDF-threshold selection, tau 0.9, capacity = budget"
     if w.drift:
         line["stages"]["drift_ms"] = dr_ms
         line["stages"]["drift_tflops"] = w.drift_flops() * H / w.heads / (dr_ms / 1e3) / 1e12

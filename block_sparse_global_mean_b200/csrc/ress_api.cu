@@ -37,6 +37,17 @@ ress_status check_shape(const ress_shape* s, Geometry* g) {
   return RESS_OK;
 }
 
+ress_status check_layout(const ress_layout* lay, Geometry* g) {
+  if (lay == nullptr) return RESS_ERR_INVALID_ARG;
+  const int t = lay->tokens_per_view, r = lay->real_tokens, sp = lay->special_tokens;
+  if (t <= 0 || t % g->block != 0 || g->n % t != 0) return RESS_ERR_INVALID_ARG;
+  if (r < 1 || r > t || sp < 0 || sp > r) return RESS_ERR_INVALID_ARG;
+  g->lay_t = t;
+  g->lay_r = r;
+  g->lay_s = sp;
+  return RESS_OK;
+}
+
 ress_status check_budget(const Geometry& g, int32_t budget) {
   if (g.nb == 0) return RESS_OK;
   return (budget >= 1 && budget <= g.nb) ? RESS_OK : RESS_ERR_INVALID_ARG;
@@ -141,6 +152,24 @@ bool make_token_map(CUtensorMap* map, const void* base, const Geometry& g, int r
   return r == CUDA_SUCCESS;
 }
 
+bool make_f32_rows_map(CUtensorMap* map, const void* base, int rows, int heads,
+                       size_t head_stride_bytes) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
+  if (encode == nullptr) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)kHeadDim, (cuuint64_t)rows, (cuuint64_t)heads};
+  const cuuint64_t strides[2] = {(cuuint64_t)kHeadDim * 4, (cuuint64_t)head_stride_bytes};
+  const cuuint32_t box[3] = {32u, 128u, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims,
+                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+             "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return r == CUDA_SUCCESS;
+}
+
 ress_status launch_cast_bf16(const float* src, __nv_bfloat16* dst, size_t count, cudaStream_t st) {
   const size_t n4 = count / 4;   // count is a multiple of 64
   if (n4 == 0) return RESS_OK;
@@ -194,6 +223,26 @@ ress_status ress_select_blocks(const ress_shape* shape, const void* q, const voi
     return RESS_ERR_INVALID_ARG;
   if (workspace_bytes < select_layout(g, with_v).total) return RESS_ERR_WORKSPACE;
   return launch_select(g, q, k, with_v ? v : nullptr, budget, lambda, idx, workspace,
+                       static_cast<cudaStream_t>(stream));
+}
+
+ress_status ress_select_blocks_layout(const ress_shape* shape, const ress_layout* layout,
+                                      const void* q, const void* k, int32_t budget,
+                                      int32_t* idx, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+  Geometry g;
+  ress_status s = check_shape(shape, &g);
+  if (s != RESS_OK) return s;
+  if ((s = check_layout(layout, &g)) != RESS_OK) return s;
+  if ((s = check_budget(g, budget)) != RESS_OK) return s;
+  if (g.nb == 0) return RESS_OK;
+  if (g.nb > kMaxBlocksSelect) return RESS_ERR_UNSUPPORTED;
+  if (!q || !k || !idx || !workspace) return RESS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(workspace) & 255u) ||
+      (reinterpret_cast<uintptr_t>(idx) & 3u))
+    return RESS_ERR_INVALID_ARG;
+  if (workspace_bytes < select_layout(g, false).total) return RESS_ERR_WORKSPACE;
+  return launch_select(g, q, k, nullptr, budget, 0.f, idx, workspace,
                        static_cast<cudaStream_t>(stream));
 }
 
@@ -269,6 +318,51 @@ ress_status ress_block_sparse_attn(const ress_shape* shape, const void* q, const
   return launch_attn(g, q, k, v, budget, idx, out, out_dtype == RESS_F32, lse, st);
 }
 
+size_t ress_attn_layout_workspace_bytes(const ress_shape* shape, const ress_layout* layout,
+                                        int32_t out_dtype) {
+  Geometry g;
+  if (check_shape(shape, &g) != RESS_OK || check_layout(layout, &g) != RESS_OK) return 0;
+  if (out_dtype != RESS_BF16 && out_dtype != RESS_F32) return 0;
+  return ress_attn_workspace_bytes(shape) + special_layout(g, out_dtype == RESS_F32).total;
+}
+
+ress_status ress_block_sparse_attn_layout(const ress_shape* shape, const ress_layout* layout,
+                                          const void* q, const void* k, const void* v,
+                                          int32_t budget, const int32_t* idx, void* out,
+                                          int32_t out_dtype, float* lse, void* workspace,
+                                          size_t workspace_bytes, void* stream) {
+  Geometry g;
+  ress_status s = check_shape(shape, &g);
+  if (s != RESS_OK) return s;
+  if ((s = check_layout(layout, &g)) != RESS_OK) return s;
+  if ((s = check_budget(g, budget)) != RESS_OK) return s;
+  if (g.nb == 0) return RESS_OK;
+  if (!q || !k || !v || !idx || !out) return RESS_ERR_INVALID_ARG;
+  if (out_dtype != RESS_BF16 && out_dtype != RESS_F32) return RESS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (reinterpret_cast<uintptr_t>(idx) & 3u) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return RESS_ERR_INVALID_ARG;
+  const size_t stage = ress_attn_workspace_bytes(shape);
+  const SpecialLayout sl = special_layout(g, out_dtype == RESS_F32);
+  if (stage + sl.total > 0) {
+    if (!workspace || workspace_bytes < stage + sl.total) return RESS_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return RESS_ERR_INVALID_ARG;
+  }
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = stage_inputs(g, q, k, v, workspace, workspace_bytes, st)) != RESS_OK) return s;
+  if ((s = launch_attn(g, q, k, v, budget, idx, out, out_dtype == RESS_F32, lse, st)) != RESS_OK)
+    return s;
+  return launch_special_rows(g, q, k, v, out, out_dtype == RESS_F32, lse,
+                             static_cast<uint8_t*>(workspace) + stage, st);
+}
+
+namespace {
+ress_status drift_checked(Geometry& g, const ress_shape* shape, const void* q, const void* k,
+                          const void* v, int32_t budget, const int32_t* idx, const float* lse,
+                          float* drift, float* set_drift, void* workspace, size_t workspace_bytes,
+                          void* stream);
+}  // namespace
+
 ress_status ress_block_drift(const ress_shape* shape, const void* q, const void* k,
                              const void* v, int32_t budget, const int32_t* idx,
                              const float* lse, float* drift, float* set_drift,
@@ -276,6 +370,29 @@ ress_status ress_block_drift(const ress_shape* shape, const void* q, const void*
   Geometry g;
   ress_status s = check_shape(shape, &g);
   if (s != RESS_OK) return s;
+  return drift_checked(g, shape, q, k, v, budget, idx, lse, drift, set_drift, workspace,
+                       workspace_bytes, stream);
+}
+
+ress_status ress_block_drift_layout(const ress_shape* shape, const ress_layout* layout,
+                                    const void* q, const void* k, const void* v, int32_t budget,
+                                    const int32_t* idx, const float* lse, float* drift,
+                                    float* set_drift, void* workspace, size_t workspace_bytes,
+                                    void* stream) {
+  Geometry g;
+  ress_status s = check_shape(shape, &g);
+  if (s != RESS_OK) return s;
+  if ((s = check_layout(layout, &g)) != RESS_OK) return s;
+  return drift_checked(g, shape, q, k, v, budget, idx, lse, drift, set_drift, workspace,
+                       workspace_bytes, stream);
+}
+
+namespace {
+ress_status drift_checked(Geometry& g, const ress_shape* shape, const void* q, const void* k,
+                          const void* v, int32_t budget, const int32_t* idx, const float* lse,
+                          float* drift, float* set_drift, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  ress_status s;
   if ((s = check_budget(g, budget)) != RESS_OK) return s;
   if (g.nb == 0) return RESS_OK;
   if (!q || !k || !v || !idx || !lse || (budget < g.nb && !drift)) return RESS_ERR_INVALID_ARG;
@@ -289,6 +406,7 @@ ress_status ress_block_drift(const ress_shape* shape, const void* q, const void*
   if ((s = stage_inputs(g, q, k, v, workspace, workspace_bytes, st)) != RESS_OK) return s;
   return launch_drift(g, q, k, v, budget, idx, lse, drift, set_drift, st);
 }
+}  // namespace
 
 ress_status ress_validate_idx(const ress_shape* shape, int32_t budget, const int32_t* idx,
                               void* stream) {

@@ -49,16 +49,30 @@ constexpr uint32_t kColO = 384;                    // O of the even / odd chunks
 
 struct AttnParams {
   DeviceError* err;
-  int n;
+  int n;          // key tokens
+  int nq;         // query tokens (rows of Q, out and lse); n except in the dense pass
   int heads;
-  int nb;
+  int nb;         // key blocks
+  int nbq;        // query blocks
   int block;
   int budget;
   int tiles_per_head;
+  int dense;      // every key block is kept for every query row (idx unused)
+  int lay_t, lay_r, lay_s;   // per-view layout (lay_t == 0: none)
   const int32_t* idx;
   void* out;
   float* lse;
 };
+
+// Sets the S columns of one 64-key sub-block beyond its valid prefix to -inf
+// (padding keys never enter the softmax).
+__device__ __forceinline__ void mask_sub_block(uint32_t (&r0)[32], uint32_t (&r1)[32], int valid) {
+#pragma unroll
+  for (int u = 0; u < 32; ++u) {
+    if (u >= valid) r0[u] = 0xFF800000u;
+    if (u + 32 >= valid) r1[u] = 0xFF800000u;
+  }
+}
 
 struct __align__(8) Ctl {
   uint64_t q_full;
@@ -227,17 +241,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_addr(&ctl->tmem_base), kTmemCols);
     tmem_relinquish();
   }
-  for (int w = threadIdx.x; w < 2 * W; w += kThreads) bmA[w] = 0u;
+  // Dense pass: every key block, for both query blocks of the tile.
+  for (int w = threadIdx.x; w < 2 * W; w += kThreads) {
+    const int ww = w < W ? w : w - W;
+    bmA[w] = p.dense ? ((ww < p.nb >> 5) ? 0xFFFFFFFFu : ((1u << (p.nb & 31)) - 1u)) : 0u;
+  }
   __syncthreads();
 
   // Kept sets of the tile's query blocks as bitmaps (duplicates collapse,
   // out-of-range entries are skipped and flagged).
-  for (int e = threadIdx.x; e < nsets * p.budget; e += kThreads) {
+  for (int e = threadIdx.x; e < (p.dense ? 0 : nsets * p.budget); e += kThreads) {
     const int s = e / p.budget;
     const int r = e - s * p.budget;
     const int qb = qb0 + s;
-    if (qb >= p.nb) continue;
-    const int j = p.idx[((size_t)h * p.nb + qb) * p.budget + r];
+    if (qb >= p.nbq) continue;
+    const int j = p.idx[((size_t)h * p.nbq + qb) * p.budget + r];
     if (j < 0 || j >= p.nb) {
       raise_device_error(p.err, RESS_ERR_BAD_INDEX, 1);
       continue;
@@ -413,8 +431,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int t0, t1;
       uint32_t m0, m1;
       chunk_info(list, n_entries, p.block, c, t0, t1, m0, m1);
-      const bool use0 = (m0 >> half) & 1u;
-      const bool use1 = (m1 >> half) & 1u;
+      // Valid (non-padding) prefix of each 64-key sub-block.
+      const int vk0 = layout_valid(p.lay_t, p.lay_r, t0, 64);
+      const int vk1 = layout_valid(p.lay_t, p.lay_r, t1, 64);
+      const bool use0 = ((m0 >> half) & 1u) && vk0 > 0;
+      const bool use1 = ((m1 >> half) & 1u) && vk1 > 0;
       if (!use0 && !use1) {
         uint32_t z[32];
 #pragma unroll
@@ -432,6 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tS + 64, r[2]);
       tmem_ld32(tS + 96, r[3]);
       tmem_ld_wait();
+      if (vk0 < 64) mask_sub_block(r[0], r[1], vk0);
+      if (vk1 < 64) mask_sub_block(r[2], r[3], vk1);
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
       if (use0) {
 #pragma unroll
@@ -514,18 +537,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Epilogue: the odd-chunk group posts its row statistics; the even-chunk
     // group merges both partial results and writes the row.
     const int tok = row0 + row;
+    const bool query_pad = !p.dense && p.lay_t != 0 && (tok % p.lay_t) >= p.lay_r;
     if (par == 1) {
       ctl->odd_m[row] = m_ref;
       ctl->odd_lr[row] = lr_sum;
       mbar_arrive(bar_merge);
     } else if (n_chunks == 0) {
-      if (tok < p.n) {
+      // No kept key: output 0, lse -inf.
+      if (tok < p.nq) {
         float zero[64];
 #pragma unroll
         for (int u = 0; u < 64; ++u) zero[u] = 0.f;
         store_row(reinterpret_cast<OutT*>(p.out) + ((size_t)tok * p.heads + h) * kHeadDim, zero,
                   0.f);
-        if (p.lse) p.lse[(size_t)h * p.n + tok] = -INFINITY;
+        if (p.lse) p.lse[(size_t)h * p.nq + tok] = -INFINITY;
       }
     } else if (ok && warp_wait(bar_o, 0, abortf, p.err, 31) &&
                warp_wait(bar_merge, 0, abortf, p.err, 33)) {
@@ -537,7 +562,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float a0 = fast_exp2(m_ref - m);    // 0 when this group never saw the row
       const float a1 = two ? fast_exp2(m1v - m) : 0.f;
       const float lr = fmaf(a1, lr1, a0 * lr_sum);
-      const float inv = 1.0f / lr;
+      // lr == 0 only when every kept key of the row is padding; a padding
+      // query (its lanes diverge only here, after the warp-wide TMEM reads)
+      // outputs 0 as well, with lse -inf.
+      const bool zero_row = query_pad || !(lr > 0.f);
+      const float inv = zero_row ? 0.f : 1.0f / lr;
       OutT* dst = reinterpret_cast<OutT*>(p.out) + ((size_t)tok * p.heads + h) * kHeadDim;
 #pragma unroll
       for (int hc = 0; hc < 2; ++hc) {
@@ -550,11 +579,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int u = 0; u < 32; ++u) {
           of[u] = a0 * __uint_as_float(oa[u]);
           if (two) of[u] = fmaf(a1, __uint_as_float(ob[u]), of[u]);
+          if (zero_row) of[u] = 0.f;
         }
-        if (tok < p.n) store_half_row(dst + 32 * hc, of, inv);
+        if (tok < p.nq) store_half_row(dst + 32 * hc, of, inv);
       }
-      if (tok < p.n && p.lse)
-        p.lse[(size_t)h * p.n + tok] = (m + __log2f(lr)) * 0.6931471805599453f;
+      if (tok < p.nq && p.lse)
+        p.lse[(size_t)h * p.nq + tok] =
+            zero_row ? -INFINITY : (m + __log2f(lr)) * 0.6931471805599453f;
     }
   }
 
@@ -588,22 +619,30 @@ ress_status launch_exp2_poly_test(const float* x, float* y, int n, cudaStream_t 
 
 bool make_token_map(CUtensorMap* map, const void* base, const Geometry& g, int rows);
 
-ress_status launch_attn(const Geometry& g, const void* q, const void* k, const void* v,
-                        int budget, const int32_t* idx, void* out, bool out_f32, float* lse,
-                        cudaStream_t st) {
+ress_status launch_attn_rows(const Geometry& g, const void* q, int64_t nq, bool dense,
+                             const void* k, const void* v, int budget, const int32_t* idx,
+                             void* out, bool out_f32, float* lse, cudaStream_t st) {
+  Geometry gq = g;
+  gq.n = nq;
   CUtensorMap tq, tk, tv;
-  if (!make_token_map(&tq, q, g, 128) || !make_token_map(&tk, k, g, 64) ||
+  if (!make_token_map(&tq, q, gq, 128) || !make_token_map(&tk, k, g, 64) ||
       !make_token_map(&tv, v, g, 64))
     return RESS_ERR_CUDA;
   AttnParams p{};
   p.err = device_error_ptr();
   if (p.err == nullptr) return RESS_ERR_CUDA;
   p.n = (int)g.n;
+  p.nq = (int)nq;
   p.heads = g.heads;
   p.nb = g.nb;
+  p.nbq = (int)(nq / g.block);
   p.block = g.block;
   p.budget = budget;
-  p.tiles_per_head = (g.block == 64) ? (g.nb + 1) / 2 : g.nb;
+  p.dense = dense ? 1 : 0;
+  p.lay_t = g.lay_t;
+  p.lay_r = g.lay_r;
+  p.lay_s = g.lay_s;
+  p.tiles_per_head = (g.block == 64) ? (p.nbq + 1) / 2 : p.nbq;
   p.idx = idx;
   p.out = out;
   p.lse = lse;
@@ -622,6 +661,12 @@ ress_status launch_attn(const Geometry& g, const void* q, const void* k, const v
     block_sparse_attn_kernel<__nv_bfloat16><<<grid, kThreads, smem, st>>>(tq, tk, tv, p);
   }
   return record_cuda(cudaGetLastError());
+}
+
+ress_status launch_attn(const Geometry& g, const void* q, const void* k, const void* v,
+                        int budget, const int32_t* idx, void* out, bool out_f32, float* lse,
+                        cudaStream_t st) {
+  return launch_attn_rows(g, q, g.n, false, k, v, budget, idx, out, out_f32, lse, st);
 }
 
 }  // namespace ress

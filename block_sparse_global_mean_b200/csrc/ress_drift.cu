@@ -57,6 +57,7 @@ struct DriftParams {
   const float* lse;
   float* drift;
   float* set_drift;
+  int lay_t, lay_r, lay_s;   // per-view layout (lay_t == 0: none)
 };
 
 struct __align__(8) Ctl {
@@ -366,7 +367,12 @@ __global__ void __launch_bounds__(kThreads, B128 ? 2 : 1)
     const uint32_t tS = tmem + kColS + lane_off;
     const float kScaleLog2 = 1.4426950408889634f * 0.125f;
     const int tok = row0 + row;
-    const float lse2 = (tok < p.n) ? p.lse[(size_t)h * p.n + tok] * 1.4426950408889634f : 0.f;
+    // Layout: only the valid, non-special queries drop anything.
+    const int pos = p.lay_t != 0 ? tok % p.lay_t : 0;
+    const bool live_q = p.lay_t == 0 || (pos < p.lay_r && pos >= p.lay_s);
+    const bool all_live = __all_sync(0xffffffffu, live_q);
+    const float lse2 =
+        (tok < p.n && live_q) ? p.lse[(size_t)h * p.n + tok] * 1.4426950408889634f : 0.f;
     const float neg_l = -lse2;
     const int sub_tid = threadIdx.x - 64;   // 0..127 among the softmax warps
     bool ok = true;
@@ -378,6 +384,8 @@ __global__ void __launch_bounds__(kThreads, B128 ? 2 : 1)
       chunk_info(list, n_entries, p.block, c, t0, t1, j0, j1, m0, m1);
       const bool use0 = (m0 >> half) & 1u;
       const bool use1 = (m1 >> half) & 1u;
+      const int vk0 = layout_valid(p.lay_t, p.lay_r, t0, 64);   // valid keys of each sub-block
+      const int vk1 = layout_valid(p.lay_t, p.lay_r, t1, 64);
       if (use0 || use1) {
         // Two halves of 64 columns; P (bf16, two per column) of half hf goes
         // to columns 32 hf .. 32 hf + 31, below the S columns still unread.
@@ -391,11 +399,26 @@ __global__ void __launch_bounds__(kThreads, B128 ? 2 : 1)
           for (int g = 0; g < 2; ++g) {
             const bool use = hf == 0 ? use0 : use1;
             uint32_t pk[16];
+            const int vk = hf == 0 ? vk0 : vk1;
+            if (use && vk == 64 && all_live) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float p0 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e]), kScaleLog2, neg_l));
-              const float p1 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e + 1]), kScaleLog2, neg_l));
-              pk[e] = use ? pack_bf16x2(p0, p1) : 0u;
+              for (int e = 0; e < 16; ++e) {
+                const float p0 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e]), kScaleLog2, neg_l));
+                const float p1 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e + 1]), kScaleLog2, neg_l));
+                pk[e] = pack_bf16x2(p0, p1);
+              }
+            } else {
+              // Layout: padding keys (columns beyond the sub-block's valid
+              // prefix) and the rows of padding and special queries add nothing.
+#pragma unroll
+              for (int e = 0; e < 16; ++e) {
+                const int col = 32 * g + 2 * e;
+                float p0 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e]), kScaleLog2, neg_l));
+                float p1 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e + 1]), kScaleLog2, neg_l));
+                if (!use || !live_q || col >= vk) p0 = 0.f;
+                if (!use || !live_q || col + 1 >= vk) p1 = 0.f;
+                pk[e] = pack_bf16x2(p0, p1);
+              }
             }
             tmem_st16(tS + 32 * hf + 16 * g, pk);
           }
@@ -551,6 +574,9 @@ ress_status launch_drift(const Geometry& g, const void* q, const void* k, const 
   p.lse = lse;
   p.drift = drift;
   p.set_drift = set_drift;
+  p.lay_t = g.lay_t;
+  p.lay_r = g.lay_r;
+  p.lay_s = g.lay_s;
   const size_t smem = drift_smem_bytes(g.nb);
   if (smem > 227 * 1024) return RESS_ERR_UNSUPPORTED;   // block lists no longer fit
   const unsigned grid = (unsigned)(g.heads * p.tiles_per_head);

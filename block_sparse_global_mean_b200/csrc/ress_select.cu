@@ -33,7 +33,22 @@ struct PoolArgs {
   float* dst[kPoolMaxTensors];
   int layout[kPoolMaxTensors];  // 0: [H][nb][64]; 1: [H][64][nb_pad] (transposed)
   int nb, nb_pad, block, heads, vpr;
+  // Extra outputs for the keys (tensor 1), written when khi != null: the
+  // pooled keys split into a tf32 high part and a tf32 low part, both
+  // [H][nb_pad][64] (key-major), the high parts of 128 evenly spaced sample
+  // keys [H][128][64] (sample t is key (t * nb) / 128), and the key norms
+  // [H][nb].
+  float* khi;
+  float* klo;
+  float* ksample;
+  float* knorm;
+  int lay_t, lay_r;   // per-view layout (lay_t == 0: none): only valid tokens are pooled
 };
+
+// float32 -> nearest tf32 (10 explicit mantissa bits), kept in a float.
+__device__ __forceinline__ float round_tf32(float x) {
+  return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
+}
 
 __device__ __forceinline__ void accum_vec(float* acc, const uint4& v, const __nv_bfloat16*) {
   const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
@@ -70,19 +85,21 @@ __global__ void __launch_bounds__(1024, 1) pool_kernel(const PoolArgs a) {
   float* dst = t == 0 ? a.dst[0] : (t == 1 ? a.dst[1] : a.dst[2]);
   const int layout = t == 0 ? a.layout[0] : (t == 1 ? a.layout[1] : a.layout[2]);
   const uint4* base = reinterpret_cast<const uint4*>(src) + (size_t)i * a.block * vpr + col;
+  // Tokens pooled: the block's valid prefix (all of it without a layout).
+  const int cnt = layout_valid(a.lay_t, a.lay_r, (long long)i * a.block, a.block);
   float acc[EPV];
 #pragma unroll
   for (int u = 0; u < EPV; ++u) acc[u] = 0.f;
   int tok = ph;
 #pragma unroll 1
-  for (; tok + 7 * phases < a.block; tok += 8 * phases) {
+  for (; tok + 7 * phases < cnt; tok += 8 * phases) {
     uint4 v[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) v[u] = __ldg(base + (size_t)(tok + u * phases) * vpr);
 #pragma unroll
     for (int u = 0; u < 8; ++u) accum_vec(acc, v[u], (const T*)nullptr);
   }
-  for (; tok < a.block; tok += phases) {
+  for (; tok < cnt; tok += phases) {
     const uint4 v = __ldg(base + (size_t)tok * vpr);
     accum_vec(acc, v, (const T*)nullptr);
   }
@@ -96,10 +113,44 @@ __global__ void __launch_bounds__(1024, 1) pool_kernel(const PoolArgs a) {
       for (int u = 0; u < EPV; ++u) acc[u] += red[(q * vpr + col) * EPV + u];
     }
   }
-  const float inv = 1.0f / (float)a.block;
+  // An empty block (no valid token) pools to zero.
+  const float inv = cnt > 0 ? 1.0f / (float)cnt : 0.f;
   const int e0 = col * EPV;           // element within the token row (H * 64)
   const int hh = e0 / kHeadDim;
   const int dd = e0 % kHeadDim;
+  if (t == 1 && a.khi != nullptr) {
+    // Lanes holding one head's 64 values: 64 / EPV consecutive lanes, all in
+    // phase 0 (the lanes of other phases have returned above).
+    constexpr int G = kHeadDim / EPV;
+    const int lane = threadIdx.x & 31;
+    const unsigned gmask = (G == 32 ? 0xffffffffu : ((1u << G) - 1u)) << (lane & ~(G - 1));
+    float v[EPV], hi[EPV], lo[EPV];
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < EPV; ++u) {
+      v[u] = acc[u] * inv;
+      hi[u] = round_tf32(v[u]);
+      lo[u] = round_tf32(v[u] - hi[u]);
+      ss = fmaf(v[u], v[u], ss);
+    }
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(gmask, ss, o);
+    const size_t krow = ((size_t)hh * a.nb_pad + i) * kHeadDim + dd;
+#pragma unroll
+    for (int u = 0; u < EPV; u += 4) {
+      *reinterpret_cast<float4*>(a.khi + krow + u) = make_float4(hi[u], hi[u + 1], hi[u + 2], hi[u + 3]);
+      *reinterpret_cast<float4*>(a.klo + krow + u) = make_float4(lo[u], lo[u + 1], lo[u + 2], lo[u + 3]);
+    }
+    if ((lane & (G - 1)) == 0) a.knorm[(size_t)hh * a.nb + i] = sqrtf(ss);
+    // Sample slots whose key is this block: t_s with (t_s * nb) / 128 == i.
+    for (int ts = (i * 128 + a.nb - 1) / a.nb; ts < 128 && (ts * a.nb) / 128 == i; ++ts) {
+      float* srow = a.ksample + ((size_t)hh * 128 + ts) * kHeadDim + dd;
+#pragma unroll
+      for (int u = 0; u < EPV; u += 4)
+        *reinterpret_cast<float4*>(srow + u) = make_float4(hi[u], hi[u + 1], hi[u + 2], hi[u + 3]);
+    }
+  }
+  if (dst == nullptr) return;
   if (layout == 0) {
     float4* o = reinterpret_cast<float4*>(dst + ((size_t)hh * a.nb + i) * kHeadDim + dd);
 #pragma unroll
@@ -154,6 +205,7 @@ struct ScoreArgs {
   float lambda;
   float tau;              // CDF threshold (cdf_counts != null)
   int32_t* cdf_counts;    // [H][nb] CDF counts, or null for the fixed budget
+  int block, lay_t, lay_r, lay_s;   // per-view layout (lay_t == 0: none)
 };
 
 // Exact selection of `budget` largest keys of a shared-memory row (one warp):
@@ -685,7 +737,7 @@ struct ScoreCfg {
 
 // Registers are capped at 128 so that four warps of one SM sub-partition fit
 // its register file (4 x 32 x 128 = 16,384).
-template <int R>
+template <int R, bool kCdf>
 __global__ void __maxnreg__(128) score_topk_kernel(const ScoreArgs a) {
   using C = ScoreCfg<R>;
   constexpr int TK = kScoreTK, TD = kScoreTD;
@@ -824,7 +876,7 @@ __global__ void __maxnreg__(128) score_topk_kernel(const ScoreArgs a) {
   uint32_t* whist = reinterpret_cast<uint32_t*>(stages) + warp * kWarpScratchStride;
   float* row = scores + (size_t)warp * rs;
   int32_t* out = a.idx + ((size_t)h * nb + i) * a.budget;
-  if (a.cdf_counts != nullptr) {
+  if constexpr (kCdf) {
     // CDF threshold: the count, then the exact top min(count, capacity) of the
     // logits (the probabilities' order), padded with the last kept block.
     // At least one unit: every row keeps at least its top block.
@@ -838,6 +890,19 @@ __global__ void __maxnreg__(128) score_topk_kernel(const ScoreArgs a) {
     for (int r = keep + lane; r < a.budget; r += 32) out[r] = last;
     if (lane == 0) a.cdf_counts[(size_t)h * nb + i] = k;
     return;
+  }
+  if (a.lay_t != 0) {
+    // Layout: an empty key block (no valid token) ranks below every other
+    // block, a key block whose valid tokens are all special ranks above
+    // (kept first, lowest index first when there are more than the budget).
+    for (int j = lane; j < nb; j += 32) {
+      const long long t0 = (long long)j * a.block;
+      const int cnt = layout_valid(a.lay_t, a.lay_r, t0, a.block);
+      const int sp = layout_valid(a.lay_t, a.lay_s, t0, a.block);
+      if (cnt == 0) row[j] = -INFINITY;
+      else if (sp == cnt) row[j] = INFINITY;
+    }
+    __syncwarp();
   }
   if (a.lambda != 0.f) {
     float m = -INFINITY;
@@ -875,26 +940,100 @@ int score_stages(int row_stride, int min_stages) {
   return 0;
 }
 
-template <int R>
-ress_status launch_score(const ScoreArgs& a0, int stages, cudaStream_t st) {
+template <int R, bool kCdf>
+ress_status launch_score_mode(const ScoreArgs& a0, int stages, cudaStream_t st) {
   ScoreArgs a = a0;
   a.tiles_per_head = (a.nb + R - 1) / R;
   a.stages = stages;
   const size_t smem = score_smem_bytes<R>(stages, a.row_stride);
   if (ress_status st_ = record_cuda(cudaFuncSetAttribute(
-          score_topk_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+          score_topk_kernel<R, kCdf>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
     return st_;
-  score_topk_kernel<R><<<a.heads * a.tiles_per_head, ScoreCfg<R>::kThreads, smem, st>>>(a);
+  score_topk_kernel<R, kCdf><<<a.heads * a.tiles_per_head, ScoreCfg<R>::kThreads, smem, st>>>(a);
   return record_cuda(cudaGetLastError());
 }
 
+// The CDF mode is a separate instantiation, so that its code does not weigh on
+// the register allocation and code layout of the fixed-budget kernel.
+template <int R>
+ress_status launch_score(const ScoreArgs& a, int stages, cudaStream_t st) {
+  return a.cdf_counts != nullptr ? launch_score_mode<R, true>(a, stages, st)
+                                 : launch_score_mode<R, false>(a, stages, st);
+}
+
+// Exact top-k of the rows that the tensor-core kernel handed over (its check
+// failed: a crowded threshold band, or a band that missed the budget-th
+// score).  A persistent grid walks the list; per row the pooled scores are
+// float32 FMA dot products over d in ascending order, scaled by the exact
+// 1/8 (the shared-memory kernel's arithmetic), with the keys read back as
+// their tf32 high + low parts, and warp 0 selects the top `budget`.
+struct FallbackArgs {
+  const float* qbar;          // [H][nb][64]
+  const float* khi;           // [H][nb_pad][64]
+  const float* klo;           // [H][nb_pad][64]
+  const int32_t* fb_count;
+  const int32_t* fb_list;
+  int32_t* idx;
+  int nb, nb_pad, budget, row_stride;
+};
+
+__global__ void __launch_bounds__(512) topk_fallback_kernel(const FallbackArgs a) {
+  extern __shared__ __align__(16) float fsm[];
+  float* row = fsm;                                  // [row_stride]
+  float* qs = row + a.row_stride;                    // [64]
+  uint32_t* scratch = reinterpret_cast<uint32_t*>(qs + kHeadDim);   // [kWarpScratchStride]
+  const int count = *a.fb_count;
+  for (int t = blockIdx.x; t < count; t += gridDim.x) {
+    const int code = a.fb_list[t];
+    const int h = code / a.nb, i = code - h * a.nb;
+    if (threadIdx.x < kHeadDim) qs[threadIdx.x] = a.qbar[((size_t)h * a.nb + i) * kHeadDim + threadIdx.x];
+    __syncthreads();
+    for (int j = threadIdx.x; j < a.nb; j += blockDim.x) {
+      const float* kh = a.khi + ((size_t)h * a.nb_pad + j) * kHeadDim;
+      const float* kl = a.klo + ((size_t)h * a.nb_pad + j) * kHeadDim;
+      float acc = 0.f;
+#pragma unroll 16
+      for (int d = 0; d < kHeadDim; ++d) acc = fmaf(qs[d], kh[d] + kl[d], acc);
+      row[j] = acc * 0.125f;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32)
+      warp_topk_row_binned(row, a.nb, a.budget, scratch,
+                           a.idx + ((size_t)h * a.nb + i) * a.budget, threadIdx.x);
+    __syncthreads();
+  }
+}
+
 }  // namespace
+
+ress_status launch_topk_fallback(const Geometry& g, int budget, int32_t* idx, uint8_t* ws,
+                                 const SelectLayout& lay, cudaStream_t st) {
+  FallbackArgs a{};
+  a.qbar = reinterpret_cast<const float*>(ws + lay.qbar);
+  a.khi = reinterpret_cast<const float*>(ws + lay.tc_khi);
+  a.klo = reinterpret_cast<const float*>(ws + lay.tc_klo);
+  a.fb_count = reinterpret_cast<const int32_t*>(ws + lay.tc_fb_count);
+  a.fb_list = reinterpret_cast<const int32_t*>(ws + lay.tc_fb_list);
+  a.idx = idx;
+  a.nb = g.nb;
+  a.nb_pad = g.nb_pad;
+  a.budget = budget;
+  a.row_stride = (g.nb + 3) & ~3;
+  const size_t smem = sizeof(float) * ((size_t)a.row_stride + kHeadDim) +
+                      sizeof(uint32_t) * kWarpScratchStride;
+  if (ress_status st_ = record_cuda(cudaFuncSetAttribute(
+          topk_fallback_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+    return st_;
+  topk_fallback_kernel<<<148, 512, smem, st>>>(a);
+  return record_cuda(cudaGetLastError());
+}
 
 SelectLayout select_layout(const Geometry& g, bool with_v) {
   SelectLayout l{};
   size_t off = 0;
   l.qbar = off;
   off += align256(sizeof(float) * (size_t)g.heads * g.nb * kHeadDim);
+  const size_t after_qbar = off;
   l.kbar_t = off;
   off += align256(sizeof(float) * (size_t)g.heads * kHeadDim * g.nb_pad);
   if (with_v) {
@@ -902,11 +1041,31 @@ SelectLayout select_layout(const Geometry& g, bool with_v) {
     off += align256(sizeof(float) * (size_t)g.heads * g.nb * kHeadDim);
     l.contrast = off;
     off += align256(sizeof(float) * (size_t)g.heads * g.nb);
-  } else {
-    l.vbar = l.contrast = 0;
+    l.total = off;
+    return l;
   }
-  l.total = off;
+  l.vbar = l.contrast = 0;
+  // Tensor-core path (lambda == 0): the key planes overlay kbar_t and beyond.
+  size_t t = after_qbar;
+  const size_t plane = align256(sizeof(float) * (size_t)g.heads * g.nb_pad * kHeadDim);
+  l.tc_khi = t;
+  t += plane;
+  l.tc_klo = t;
+  t += plane;
+  l.tc_ksample = t;
+  t += align256(sizeof(float) * (size_t)g.heads * 128 * kHeadDim);
+  l.tc_knorm = t;
+  t += align256(sizeof(float) * (size_t)g.heads * g.nb);
+  l.tc_fb_count = t;
+  t += 256;
+  l.tc_fb_list = t;
+  t += align256(sizeof(int32_t) * (size_t)g.heads * g.nb);
+  l.total = off > t ? off : t;
   return l;
+}
+
+bool select_uses_tc(const Geometry& g, int budget, bool with_v, bool cdf) {
+  return !with_v && !cdf && g.lay_t == 0 && budget < g.nb && g.nb <= kMaxBlocksTc;
 }
 
 ress_status launch_select(const Geometry& g, const void* q, const void* k, const void* v,
@@ -920,14 +1079,23 @@ ress_status launch_select(const Geometry& g, const void* q, const void* k, const
   float* vbar = with_v ? reinterpret_cast<float*>(w + lay.vbar) : nullptr;
   float* contrast = with_v ? reinterpret_cast<float*>(w + lay.contrast) : nullptr;
 
+  const bool tc = select_uses_tc(g, budget, with_v, cdf != nullptr);
   PoolArgs pa{};
   pa.src[0] = q;  pa.dst[0] = qbar;   pa.layout[0] = 0;
-  pa.src[1] = k;  pa.dst[1] = kbar_t; pa.layout[1] = 1;
+  pa.src[1] = k;  pa.dst[1] = tc ? nullptr : kbar_t; pa.layout[1] = 1;
   pa.src[2] = v;  pa.dst[2] = vbar;   pa.layout[2] = 0;
+  if (tc) {
+    pa.khi = reinterpret_cast<float*>(w + lay.tc_khi);
+    pa.klo = reinterpret_cast<float*>(w + lay.tc_klo);
+    pa.ksample = reinterpret_cast<float*>(w + lay.tc_ksample);
+    pa.knorm = reinterpret_cast<float*>(w + lay.tc_knorm);
+  }
   pa.nb = g.nb;
   pa.nb_pad = g.nb_pad;
   pa.block = g.block;
   pa.heads = g.heads;
+  pa.lay_t = g.lay_t;
+  pa.lay_r = g.lay_r;
   const int epv = g.f32 ? 4 : 8;
   pa.vpr = g.heads * kHeadDim / epv;
   const int phases = pa.vpr >= 256 ? 1 : 256 / pa.vpr;
@@ -944,6 +1112,10 @@ ress_status launch_select(const Geometry& g, const void* q, const void* k, const
     contrast_kernel<<<(warps + 7) / 8, 256, 0, st>>>(vbar, contrast, g.heads, g.nb);
     if (ress_status st_ = record_cuda(cudaGetLastError())) return st_;
   }
+  if (tc) {
+    if (ress_status st_ = launch_topk_tc(g, budget, idx, w, lay, st)) return st_;
+    return launch_topk_fallback(g, budget, idx, w, lay, st);
+  }
   ScoreArgs sa{};
   sa.err = device_error_ptr();
   if (sa.err == nullptr) return RESS_ERR_CUDA;
@@ -958,6 +1130,10 @@ ress_status launch_select(const Geometry& g, const void* q, const void* k, const
   sa.lambda = lambda;
   sa.tau = cdf ? cdf->tau : 0.f;
   sa.cdf_counts = cdf ? cdf->counts : nullptr;
+  sa.block = g.block;
+  sa.lay_t = g.lay_t;
+  sa.lay_r = g.lay_r;
+  sa.lay_s = g.lay_s;
   sa.row_stride = (g.nb + 3) & ~3;
   // Sixteen rows per CTA while at least four stages fit next to the score rows
   // (nb <= 2,304), else eight.  The stage ring also holds the top-k scratch of

@@ -41,6 +41,11 @@ class ress_shape(ctypes.Structure):
                 ("block", ctypes.c_int32), ("dtype", ctypes.c_int32)]
 
 
+class ress_layout(ctypes.Structure):
+    _fields_ = [("tokens_per_view", ctypes.c_int32), ("real_tokens", ctypes.c_int32),
+                ("special_tokens", ctypes.c_int32)]
+
+
 _P = ctypes.c_void_p
 _SHAPE = ctypes.POINTER(ress_shape)
 
@@ -70,6 +75,18 @@ lib.ress_last_cuda_error.restype = ctypes.c_char_p
 lib.ress_last_cuda_error.argtypes = []
 lib.ress_test_exp2.restype = ctypes.c_int
 lib.ress_test_exp2.argtypes = [_P, _P, ctypes.c_int32, _P]
+_LAYOUT = ctypes.POINTER(ress_layout)
+lib.ress_select_blocks_layout.restype = ctypes.c_int
+lib.ress_select_blocks_layout.argtypes = [_SHAPE, _LAYOUT, _P, _P, ctypes.c_int32, _P, _P,
+                                          ctypes.c_size_t, _P]
+lib.ress_attn_layout_workspace_bytes.restype = ctypes.c_size_t
+lib.ress_attn_layout_workspace_bytes.argtypes = [_SHAPE, _LAYOUT, ctypes.c_int32]
+lib.ress_block_sparse_attn_layout.restype = ctypes.c_int
+lib.ress_block_sparse_attn_layout.argtypes = [_SHAPE, _LAYOUT, _P, _P, _P, ctypes.c_int32, _P, _P,
+                                              ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]
+lib.ress_block_drift_layout.restype = ctypes.c_int
+lib.ress_block_drift_layout.argtypes = [_SHAPE, _LAYOUT, _P, _P, _P, ctypes.c_int32, _P, _P, _P,
+                                        _P, _P, ctypes.c_size_t, _P]
 lib.ress_validate_idx.restype = ctypes.c_int
 lib.ress_validate_idx.argtypes = [_SHAPE, ctypes.c_int32, _P, _P]
 lib.ress_check_device_errors.restype = ctypes.c_int
@@ -319,6 +336,107 @@ def ress_block_drift(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: tor
                                   0 if workspace is None else workspace.numel(),
                                   _stream_ptr(stream, q.device))
     _check(status, "ress_block_drift")
+    return drift, set_drift
+
+
+def _layout(layout) -> ress_layout:
+    """(tokens_per_view, real_tokens, special_tokens) -> ress_layout."""
+    t, r, sp = (int(x) for x in layout)
+    return ress_layout(t, r, sp)
+
+
+def ress_select_blocks_layout(q: torch.Tensor, k: torch.Tensor, budget: int, block: int, layout,
+                              idx: Optional[torch.Tensor] = None,
+                              workspace: Optional[torch.Tensor] = None,
+                              stream: Optional[torch.cuda.Stream] = None) -> torch.Tensor:
+    """Stage 1 with a per-view layout (tokens_per_view, real_tokens,
+    special_tokens): returns idx [H, nb, budget] int32."""
+    _check_inputs(q, k)
+    sh = _shape_of(q, block)
+    lay = _layout(layout)
+    n, h = q.shape[0], q.shape[1]
+    nb = n // block
+    if idx is None:
+        idx = torch.empty((h, nb, budget), dtype=torch.int32, device=q.device)
+    _check_buffer(idx, (h, nb, budget), torch.int32, q.device, "idx")
+    _check_workspace(workspace, q.device)
+    need = int(lib.ress_select_workspace_bytes(ctypes.byref(sh), ctypes.c_float(0.0)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    status = _on(q.device, lib.ress_select_blocks_layout, ctypes.byref(sh), ctypes.byref(lay),
+                 _ptr(q), _ptr(k), int(budget), _ptr(idx), _ptr(workspace), workspace.numel(),
+                 _stream_ptr(stream, q.device))
+    _check(status, "ress_select_blocks_layout")
+    return idx
+
+
+def ress_block_sparse_attn_layout(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                                  idx: torch.Tensor, block: int, layout,
+                                  out: Optional[torch.Tensor] = None,
+                                  lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+                                  workspace: Optional[torch.Tensor] = None,
+                                  stream: Optional[torch.cuda.Stream] = None,
+                                  out_dtype: Optional[torch.dtype] = None
+                                  ) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Stage 2 with a per-view layout: returns (out [N, H, 64], lse [H, N])."""
+    _check_inputs(q, k, v)
+    sh = _shape_of(q, block)
+    lay = _layout(layout)
+    n, h = q.shape[0], q.shape[1]
+    budget = _check_idx(idx, h, n // block, q.device)
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or q.dtype, device=q.device)
+    out_code = RESS_F32 if out.dtype == torch.float32 else (
+        RESS_BF16 if out.dtype == torch.bfloat16 else None)
+    if out_code is None:
+        raise TypeError(f"unsupported output dtype {out.dtype}")
+    _check_buffer(out, q.shape, out.dtype, q.device, "out")
+    if lse is None and want_lse:
+        lse = torch.empty((h, n), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _check_buffer(lse, (h, n), torch.float32, q.device, "lse")
+    _check_workspace(workspace, q.device)
+    need = int(lib.ress_attn_layout_workspace_bytes(ctypes.byref(sh), ctypes.byref(lay), out_code))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    status = _on(q.device, lib.ress_block_sparse_attn_layout, ctypes.byref(sh), ctypes.byref(lay),
+                 _ptr(q), _ptr(k), _ptr(v), int(budget), _ptr(idx), _ptr(out), out_code,
+                 _ptr(lse), _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                 _stream_ptr(stream, q.device))
+    _check(status, "ress_block_sparse_attn_layout")
+    return out, lse
+
+
+def ress_block_drift_layout(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, idx: torch.Tensor,
+                            lse: torch.Tensor, block: int, layout,
+                            drift: Optional[torch.Tensor] = None,
+                            set_drift: Optional[torch.Tensor] = None,
+                            workspace: Optional[torch.Tensor] = None,
+                            stream: Optional[torch.cuda.Stream] = None
+                            ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Stage 3 with a per-view layout: returns (drift [H, nb, nb - budget], set_drift [H, nb])."""
+    _check_inputs(q, k, v)
+    sh = _shape_of(q, block)
+    lay = _layout(layout)
+    n, h = q.shape[0], q.shape[1]
+    nb = n // block
+    budget = _check_idx(idx, h, nb, q.device)
+    _check_buffer(lse, (h, n), torch.float32, q.device, "lse")
+    if drift is None:
+        drift = torch.empty((h, nb, max(nb - budget, 0)), dtype=torch.float32, device=q.device)
+    if set_drift is None:
+        set_drift = torch.empty((h, nb), dtype=torch.float32, device=q.device)
+    _check_buffer(drift, (h, nb, max(nb - budget, 0)), torch.float32, q.device, "drift")
+    _check_buffer(set_drift, (h, nb), torch.float32, q.device, "set_drift")
+    _check_workspace(workspace, q.device)
+    need = int(lib.ress_attn_workspace_bytes(ctypes.byref(sh)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    status = _on(q.device, lib.ress_block_drift_layout, ctypes.byref(sh), ctypes.byref(lay),
+                 _ptr(q), _ptr(k), _ptr(v), int(budget), _ptr(idx), _ptr(lse),
+                 _ptr(drift) if drift.numel() else None, _ptr(set_drift), _ptr(workspace),
+                 0 if workspace is None else workspace.numel(), _stream_ptr(stream, q.device))
+    _check(status, "ress_block_drift_layout")
     return drift, set_drift
 
 

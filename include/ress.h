@@ -77,6 +77,25 @@ typedef struct {
   int32_t dtype;    /* ress_dtype of q, k and v */
 } ress_shape;
 
+/*
+ * Per-view layout of the concatenated sequence, for the layout-aware entry
+ * points (VASC 4.2 and A.5: camera and register queries keep dense
+ * attention, key blocks made only of special tokens are always kept, and
+ * padding takes no part in pooling or attention).  Every view occupies
+ * tokens_per_view consecutive tokens; its positions 0 .. real_tokens - 1
+ * carry data and the rest is padding; positions 0 .. special_tokens - 1 are
+ * the special (camera, register) tokens.  Requirements: tokens_per_view a
+ * multiple of the block size and a divisor of N, 1 <= real_tokens <=
+ * tokens_per_view, 0 <= special_tokens <= real_tokens.  A VGGT view is
+ * {1408, 1374, 5}: 1 camera + 4 register + 37 x 37 patch tokens, padded to
+ * 22 blocks of 64.
+ */
+typedef struct {
+  int32_t tokens_per_view;
+  int32_t real_tokens;
+  int32_t special_tokens;
+} ress_layout;
+
 /* Library version, (major << 16) | minor. */
 int ress_version(void);
 
@@ -85,10 +104,17 @@ const char* ress_status_string(ress_status status);
 
 /*
  * Workspace bytes that ress_select_blocks needs for `shape` and `lambda`
- * (0 if the shape is invalid).  Layout, all float32, each array 256-byte
- * aligned, in this order: Qbar [H][nb][64], Kbar^T [H][64][nb_pad],
- * Vbar [H][nb][64] (lambda > 0 only), contrast [H][nb] (lambda > 0 only),
- * with nb_pad = nb rounded up to 256.
+ * (0 if the shape is invalid).  Layout, each array 256-byte aligned, with
+ * nb_pad = nb rounded up to 256:
+ *   - lambda == 0, budget < nb <= 2304 (the tensor-core selection):
+ *     Qbar [H][nb][64] f32, then the pooled keys split into tf32 high and low
+ *     parts Khi, Klo [H][nb_pad][64] f32, the high parts of 128 evenly spaced
+ *     sample keys [H][128][64], the key norms [H][nb] f32, one int32 count
+ *     (in a 256-byte slot) and a row list [H][nb] int32;
+ *   - otherwise (and for ress_select_blocks_cdf): Qbar [H][nb][64],
+ *     Kbar^T [H][64][nb_pad], then Vbar [H][nb][64] and contrast [H][nb]
+ *     when lambda > 0, all float32.
+ * The size returned covers both layouts when lambda == 0.
  */
 size_t ress_select_workspace_bytes(const ress_shape* shape, float lambda);
 
@@ -175,6 +201,22 @@ ress_status ress_select_blocks_cdf(const ress_shape* shape, const void* q, const
                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Stage 1 with a per-view layout (VASC 4.2 and A.5).  As ress_select_blocks
+ * with lambda = 0, except that a block's pooled mean is over its valid
+ * (non-padding) tokens only, a key block without a valid token (it pools to
+ * zero) ranks below every other block, and a key block whose valid tokens are
+ * all special ranks above every other block (such blocks are kept first,
+ * lowest index first if there are more of them than the budget).
+ *
+ *   layout     as described at ress_layout.
+ *   workspace  ress_select_workspace_bytes(shape, 0) bytes.
+ */
+ress_status ress_select_blocks_layout(const ress_shape* shape, const ress_layout* layout,
+                                      const void* q, const void* k, int32_t budget,
+                                      int32_t* idx, void* workspace, size_t workspace_bytes,
+                                      void* stream);
+
+/*
  * Workspace bytes that ress_block_sparse_attn and ress_block_drift need:
  * 0 for bf16 inputs; 3 * N * H * 64 * 2 for float32 inputs (bf16 copies of
  * q, k and v).
@@ -210,6 +252,32 @@ ress_status ress_block_sparse_attn(const ress_shape* shape, const void* q, const
                                    const void* v, int32_t budget, const int32_t* idx,
                                    void* out, int32_t out_dtype, float* lse, void* workspace,
                                    size_t workspace_bytes, void* stream);
+
+/*
+ * Workspace bytes of ress_block_sparse_attn_layout: the float32 staging of
+ * ress_attn_workspace_bytes (float32 inputs only), then the special rows'
+ * gathered queries, outputs and lse (0 bytes when special_tokens == 0).
+ * out_dtype as for the call.  0 if the shape or layout is invalid.
+ */
+size_t ress_attn_layout_workspace_bytes(const ress_shape* shape, const ress_layout* layout,
+                                        int32_t out_dtype);
+
+/*
+ * Stage 2 with a per-view layout (VASC 4.2 and A.5).  As
+ * ress_block_sparse_attn, except that
+ *   - padding keys never enter a softmax;
+ *   - a padding query row writes 0 and lse -inf (so does a row whose kept
+ *     blocks hold no valid key);
+ *   - a special query (the first special_tokens tokens of each view) attends
+ *     densely to every valid key of the sequence, whatever idx says.
+ *   workspace  ress_attn_layout_workspace_bytes(shape, layout, out_dtype)
+ *              bytes, 256-byte aligned (NULL when that is 0).
+ */
+ress_status ress_block_sparse_attn_layout(const ress_shape* shape, const ress_layout* layout,
+                                          const void* q, const void* k, const void* v,
+                                          int32_t budget, const int32_t* idx, void* out,
+                                          int32_t out_dtype, float* lse, void* workspace,
+                                          size_t workspace_bytes, void* stream);
 
 /*
  * Stage 3: drift of the dropped blocks (ReSS Abstract and Fig. 3: the drift
@@ -254,6 +322,19 @@ ress_status ress_block_drift(const ress_shape* shape, const void* q, const void*
  */
 ress_status ress_validate_idx(const ress_shape* shape, int32_t budget, const int32_t* idx,
                               void* stream);
+
+/*
+ * Stage 3 with a per-view layout (VASC 4.2 and A.5).  As ress_block_drift,
+ * except that only valid keys enter a contribution and only the valid,
+ * non-special queries count: the rows of padding and special queries (which
+ * attend densely and drop nothing) of every C_j are zero.  lse comes from
+ * ress_block_sparse_attn_layout with the same idx.
+ */
+ress_status ress_block_drift_layout(const ress_shape* shape, const ress_layout* layout,
+                                    const void* q, const void* k, const void* v, int32_t budget,
+                                    const int32_t* idx, const float* lse, float* drift,
+                                    float* set_drift, void* workspace, size_t workspace_bytes,
+                                    void* stream);
 
 /*
  * Synchronises `stream`, then reports and clears the device error flag that

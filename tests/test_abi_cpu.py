@@ -137,12 +137,17 @@ def test_attention_and_drift_reject_bad_arguments_on_the_host(ress):
 
 def test_workspace_queries(ress):
     import torch
-    # bf16, 100 views x 1,408 tokens, H=16, B=64, lambda=0: Qbar + Kbar^T (nb_pad 2304)
+    # bf16, 100 views x 1,408 tokens, H=16, B=64 (nb_pad 2304).  lambda=0: Qbar,
+    # then the larger of Kbar^T and the tensor-core arrays (Khi, Klo, 128
+    # sample keys, key norms, a count slot, a row list).
     n, h, nb = 140800, 16, 2200
     got = ress.select_workspace_bytes(n, h, 64, torch.bfloat16, 0.0)
-    assert got == 4 * h * nb * 64 + 4 * h * 64 * 2304
+    qbar = 4 * h * nb * 64
+    tc = 2 * 4 * h * 2304 * 64 + 4 * h * 128 * 64 + 4 * h * nb + 256 + 4 * h * nb
+    assert got == qbar + max(4 * h * 64 * 2304, tc)
+    # lambda > 0: Qbar + Kbar^T + Vbar + contrast
     with_v = ress.select_workspace_bytes(n, h, 64, torch.bfloat16, 0.5)
-    assert with_v == got + 4 * h * nb * 64 + 4 * h * nb
+    assert with_v == qbar + 4 * h * 64 * 2304 + 4 * h * nb * 64 + 4 * h * nb
     assert ress.attn_workspace_bytes(n, h, 64, torch.bfloat16) == 0
     assert ress.attn_workspace_bytes(512, 2, 64, torch.float32) == 3 * 512 * 2 * 64 * 2
     assert ress.lib.ress_select_workspace_bytes(None, ctypes.c_float(0.0)) == 0
@@ -235,3 +240,33 @@ def test_noalloc_rejects_problems_beyond_its_fixed_scratch(ress):
     assert ress.lib.ress_select_blocks_noalloc(ctypes.byref(big), FAKE, FAKE, None, 0,
                                                ctypes.c_float(0.0), FAKE, None) \
         == ress.RESS_ERR_INVALID_ARG
+
+
+@no_gpu_only
+def test_layout_entry_points_reject_bad_layouts_on_the_host(ress):
+    lib = ress.lib
+    sh = _shape(ress, n=1024, heads=2, block=64)                  # 1,024 tokens
+    bad = [ress.ress_layout(0, 1, 0), ress.ress_layout(96, 90, 5),  # not a multiple of the block
+           ress.ress_layout(384, 300, 5),                          # does not divide N
+           ress.ress_layout(256, 0, 0), ress.ress_layout(256, 257, 0),
+           ress.ress_layout(256, 200, 201), ress.ress_layout(256, 200, -1)]
+    for lay in bad:
+        assert lib.ress_select_blocks_layout(ctypes.byref(sh), ctypes.byref(lay), FAKE, FAKE, 4,
+                                             FAKE, FAKE_WS, 1 << 30, None) == ress.RESS_ERR_INVALID_ARG
+        assert lib.ress_block_sparse_attn_layout(ctypes.byref(sh), ctypes.byref(lay), FAKE, FAKE,
+                                                 FAKE, 4, FAKE, FAKE, 0, None, FAKE_WS, 1 << 30,
+                                                 None) == ress.RESS_ERR_INVALID_ARG
+        assert lib.ress_block_drift_layout(ctypes.byref(sh), ctypes.byref(lay), FAKE, FAKE, FAKE,
+                                           4, FAKE, FAKE, FAKE, None, None, 0,
+                                           None) == ress.RESS_ERR_INVALID_ARG
+        assert lib.ress_attn_layout_workspace_bytes(ctypes.byref(sh), ctypes.byref(lay), 0) == 0
+    assert lib.ress_select_blocks_layout(ctypes.byref(sh), None, FAKE, FAKE, 4, FAKE, FAKE_WS,
+                                         1 << 30, None) == ress.RESS_ERR_INVALID_ARG
+    good = ress.ress_layout(256, 200, 5)
+    # 4 views x 5 special rows -> 128 gathered rows: bf16 queries and output, float32 lse
+    assert lib.ress_attn_layout_workspace_bytes(ctypes.byref(sh), ctypes.byref(good), 0) == \
+        128 * 2 * 64 * 2 * 2 + 128 * 2 * 4
+    none = ress.ress_layout(256, 200, 0)
+    assert lib.ress_attn_layout_workspace_bytes(ctypes.byref(sh), ctypes.byref(none), 0) == 0
+    assert lib.ress_select_blocks_layout(ctypes.byref(sh), ctypes.byref(good), FAKE, FAKE, 4,
+                                         FAKE, FAKE_WS, 16, None) == ress.RESS_ERR_WORKSPACE

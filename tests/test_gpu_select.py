@@ -27,9 +27,10 @@ def _select(ress, q, k, v, budget, lam, block, **kw):
     return ress.ress_select_blocks(q, k, v, budget, lam, block, idx=idx, **kw)
 
 
-def _workspace_views(ws, H, nb, with_v):
-    """Qbar [H][nb][64], Kbar^T [H][64][nb_pad], Vbar, contrast: the layout
-    include/ress.h gives for the selection workspace."""
+def _workspace_views(ws, H, nb, with_v, tc):
+    """Qbar [H][nb][64] and the pooled keys as [H][nb][64] (from Kbar^T, or
+    from the tf32 high + low planes of the tensor-core layout), Vbar and the
+    contrast: the layouts include/ress.h gives for the selection workspace."""
     fl = ws.view(torch.float32)
     nb_pad = (nb + 255) // 256 * 256
 
@@ -39,14 +40,19 @@ def _workspace_views(ws, H, nb, with_v):
     off = 0
     qbar = fl[off:off + H * nb * 64].view(H, nb, 64)
     off += up(H * nb * 64 * 4)
-    kbar_t = fl[off:off + H * 64 * nb_pad].view(H, 64, nb_pad)[:, :, :nb]
+    if tc:
+        plane = up(H * nb_pad * 64 * 4)
+        khi = fl[off:off + H * nb_pad * 64].view(H, nb_pad, 64)[:, :nb]
+        klo = fl[off + plane:off + plane + H * nb_pad * 64].view(H, nb_pad, 64)[:, :nb]
+        return qbar, khi.double() + klo.double(), None, None
+    kbar = fl[off:off + H * 64 * nb_pad].view(H, 64, nb_pad)[:, :, :nb].transpose(1, 2)
     off += up(H * 64 * nb_pad * 4)
     vbar = contrast = None
     if with_v:
         vbar = fl[off:off + H * nb * 64].view(H, nb, 64)
         off += up(H * nb * 64 * 4)
         contrast = fl[off:off + H * nb].view(H, nb)
-    return qbar, kbar_t, vbar, contrast
+    return qbar, kbar, vbar, contrast
 
 
 @pytest.mark.parametrize("name", ["tiny", "vggt8", "views32"])
@@ -58,10 +64,12 @@ def test_pooled_means_and_contrast_match_oracle(name, ress_gpu, wcache):
     ws = torch.full((need,), 0xFF, dtype=torch.uint8, device="cuda")   # NaN-filled floats
     _select(ress_gpu, q, k, v if w.lam else None, w.budget, w.lam, w.block, workspace=ws)
     _check_errors(ress_gpu)
-    qbar, kbar_t, vbar, contrast = _workspace_views(ws, H, nb, bool(w.lam))
+    tc = w.lam == 0 and w.budget < nb <= 2304          # the tensor-core selection's layout
+    qbar, kbar, vbar, contrast = _workspace_views(ws, H, nb, bool(w.lam), tc)
     np.testing.assert_allclose(np64(qbar), oracle.pool_blocks(np64(q), w.block), rtol=2e-6, atol=2e-6)
-    np.testing.assert_allclose(np64(kbar_t).transpose(0, 2, 1), oracle.pool_blocks(np64(k), w.block),
-                               rtol=2e-6, atol=2e-6)
+    # tf32 high + low parts hold a float32 value to about 2^-22 relative
+    np.testing.assert_allclose(np64(kbar), oracle.pool_blocks(np64(k), w.block),
+                               rtol=2e-6 if not tc else 4e-6, atol=2e-6)
     if w.lam:
         ref_vbar = oracle.pool_blocks(np64(v), w.block)
         np.testing.assert_allclose(np64(vbar), ref_vbar, rtol=2e-6, atol=2e-6)
