@@ -470,3 +470,95 @@ def drift_layout_block(q, k, v, kept: Sequence[int], lse_blk, h: int, i: int, bl
     drift = np.sqrt((contrib * contrib).sum(axis=(1, 2)))
     total = contrib.sum(axis=0)
     return drift, float(np.sqrt((total * total).sum()))
+
+
+# ---------------------------------------------------------------------------
+# ReSS: drift-based selection with iterative residual restoration (pooled)
+# ---------------------------------------------------------------------------
+
+def pooled_contributions(q, k, v, block: int) -> np.ndarray:
+    """c[h, i, j, :] = p[h, i, j] * Vbar[h, j]: what key block j adds to the
+    pooled output of query block i, with p the pooled probabilities of
+    stage 1.
+
+    ReSS measures the shift each block leaves in the residual stream when it
+    is masked (ReSS, Fig. 1 and Fig. 3(a)).  Reading: at block granularity,
+    the pooled query of block i attends to key block j with its pooled
+    probability, and block j's values enter as their mean, so block j's
+    contribution is p_ij * Vbar_j.
+    """
+    sc = selection_scores(q, k, None, block, 0.0)
+    vbar = pool_blocks(v, block)
+    return sc["probs"][..., None] * vbar[:, None, :, :]
+
+
+def drop_set_drift(contrib_row, kept: Sequence[int]) -> float:
+    """J(D) = || sum_{j in D} c_j ||_2 over the drop set D (the complement of
+    `kept`): the drift of a drop set depends on the directions of the
+    contributions, not only on their sizes (ReSS, Abstract)."""
+    c = _f64(contrib_row)
+    drop = dropped_blocks(kept, c.shape[0])
+    return float(np.linalg.norm(c[drop].sum(axis=0)))
+
+
+def restore_row(contrib_row, budget: int, rounds: int, cand: int = 8):
+    """Drift-based selection of one (head, query block) row.
+
+    1. Drift score d_j = ||c_j||_2; the initial kept set is the `budget`
+       blocks of largest drift score, ties to the lower index (ReSS, Fig. 3(b):
+       the blocks with the highest scores form the initial selected set).
+    2. Up to `rounds` restoration rounds, each one budget-preserving swap that
+       reduces the drift J of the drop set (ReSS, Fig. 3(c)).  Reading of the
+       swap rule (the pages do not give it): with T = sum_{j in D} c_j,
+         - the candidates to restore (leave D) are the `cand` dropped blocks of
+           largest gain 2 <T, c_b> - ||c_b||^2 (ties: lower index),
+         - the candidates to drop (enter D) are the `cand` kept blocks of
+           smallest cost 2 <T, c_a> + ||c_a||^2 (ties: lower index),
+         - among those pairs the one of smallest ||T - c_b + c_a|| is taken
+           (ties: lower b, then lower a), and the round swaps a and b if that
+           is strictly below J; otherwise restoration stops.
+    3. Track-best: the kept set of smallest J over the initial set and every
+       round (ReSS, Table S3).  Every accepted swap lowers J, so it is the
+       last one.
+    Returns (kept blocks ascending, J of the initial set, J of the result).
+    """
+    c = _f64(contrib_row)
+    nb = c.shape[0]
+    score = np.sqrt((c * c).sum(axis=1))
+    order = np.argsort(-score, kind="stable")
+    kept = set(order[:budget].tolist())
+    j0 = drop_set_drift(c, sorted(kept))
+    best = (j0, sorted(kept))
+    for _ in range(rounds):
+        drop = [j for j in range(nb) if j not in kept]
+        if not drop or not kept:
+            break
+        t = c[drop].sum(axis=0)
+        jcur = float(np.linalg.norm(t))
+        gain = {b: 2.0 * (t @ c[b]) - c[b] @ c[b] for b in drop}
+        cost = {a: 2.0 * (t @ c[a]) + c[a] @ c[a] for a in kept}
+        out = sorted(drop, key=lambda b: (-gain[b], b))[:cand]
+        inn = sorted(kept, key=lambda a: (cost[a], a))[:cand]
+        pairs = sorted(((float(np.linalg.norm(t - c[b] + c[a])), b, a) for b in out for a in inn))
+        jnew, b, a = pairs[0]
+        if not jnew < jcur:
+            break
+        kept.remove(a)
+        kept.add(b)
+        if jnew < best[0]:
+            best = (jnew, sorted(kept))
+    return np.asarray(best[1], dtype=np.int32), j0, best[0]
+
+
+def select_blocks_restore(q, k, v, block: int, budget: int, rounds: int, cand: int = 8):
+    """ReSS-style selection of every row: idx [H, nb, budget] int32 ascending,
+    and J [H, nb] of the initial and of the restored drop sets."""
+    contrib = pooled_contributions(q, k, v, block)
+    h_count, nb = contrib.shape[:2]
+    idx = np.zeros((h_count, nb, budget), dtype=np.int32)
+    j_init = np.zeros((h_count, nb))
+    j_final = np.zeros((h_count, nb))
+    for h in range(h_count):
+        for i in range(nb):
+            idx[h, i], j_init[h, i], j_final[h, i] = restore_row(contrib[h, i], budget, rounds, cand)
+    return idx, j_init, j_final

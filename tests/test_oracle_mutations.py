@@ -57,6 +57,19 @@ MUTATIONS = {
         ("toks = toks[valid[toks]]", "toks = toks"),
     "empty key blocks ranked like the others":
         ("rank[:, :, empty] = -np.inf", "rank[:, :, empty] = rank[:, :, empty]"),
+    "restoration accepts swaps that raise J":
+        ("        if not jnew < jcur:\n            break", "        if jnew > jcur + 1e30:\n            break"),
+    "pooled contribution without the probability":
+        ("return sc[\"probs\"][..., None] * vbar[:, None, :, :]",
+         "return 0.0 * sc[\"probs\"][..., None] + vbar[:, None, :, :]"),
+    "drop-set drift as the sum of magnitudes":
+        ("return float(np.linalg.norm(c[drop].sum(axis=0)))",
+         "return float(np.linalg.norm(c[drop], axis=1).sum())"),
+    "initial set of lowest drift score":
+        ("order = np.argsort(-score, kind=\"stable\")", "order = np.argsort(score, kind=\"stable\")"),
+    "restoration candidates by the wrong sign":
+        ("out = sorted(drop, key=lambda b: (-gain[b], b))[:cand]",
+         "out = sorted(drop, key=lambda b: (gain[b], b))[:cand]"),
     "a causal mask over the kept tokens":
         ("s = (q_blk @ keys.T) / math.sqrt(d)\n    m = s.max",
          "s = (q_blk @ keys.T) / math.sqrt(d)\n    s = s + np.triu(np.full(s.shape, -np.inf), 1)\n    m = s.max"),

@@ -611,3 +611,116 @@ def test_layout_drift_reconstructs_dense_attention_over_valid_keys():
     o, l = oracle.sparse_attention_layout_block(q, k, v, idx2[0, 0], 0, 0, B, vq, sq)
     dr, jv = oracle.drift_layout_block(q, k, v, idx2[0, 0], l, 0, 0, B, vq, sq)
     assert dr.shape[0] > 0 and (dr == 0).all() and jv == 0.0
+
+
+# --------------------------------------------------------------------------
+# ReSS drift-based selection with restoration (pooled contributions)
+# --------------------------------------------------------------------------
+
+def test_pooled_contribution_is_probability_times_pooled_value():
+    w, q, k, v = _tiny_inputs()
+    c = oracle.pooled_contributions(q, k, v, w.block)
+    B = w.block
+    tq, tk, tv = (torch.tensor(x) for x in (q, k, v))
+    nb = tq.shape[0] // B
+    qb = tq.view(nb, B, *tq.shape[1:]).mean(1)      # [nb, H, d]
+    kb = tk.view(nb, B, *tk.shape[1:]).mean(1)
+    vb = tv.view(nb, B, *tv.shape[1:]).mean(1)
+    for h in range(tq.shape[1]):
+        p = torch.softmax(qb[:, h] @ kb[:, h].T / 8.0, dim=-1)      # [nb, nb]
+        ref = p[:, :, None] * vb[None, :, h]
+        assert np.allclose(c[h], ref.numpy(), atol=1e-14)
+
+
+def test_restoration_closed_form_two_rounds():
+    # Four blocks in d = 2, budget 2.  Drift scores 3, 2.9, 1, 1 keep {0, 1},
+    # so D = {2, 3} and J = 2.  Round 1: the best swap restores block 2 and
+    # drops block 1 (J = 1.9; restoring 3 instead ties and loses on index).
+    # Round 2: restore 3, drop 0: D = {0, 1}, J = |3 - 2.9| = 0.1, which no
+    # further swap improves; it is also the best of all six drop sets.
+    c = np.array([[3.0, 0.0], [-2.9, 0.0], [1.0, 0.0], [1.0, 0.0]])
+    kept, j0, j = oracle.restore_row(c, 2, rounds=1)
+    assert kept.tolist() == [0, 2] and j0 == 2.0 and abs(j - 1.9) < 1e-12
+    kept, j0, j = oracle.restore_row(c, 2, rounds=4)
+    assert kept.tolist() == [2, 3] and abs(j - 0.1) < 1e-12
+    best = min(abs(c[list(set(range(4)) - set(s))].sum(0)[0])
+               for s in itertools.combinations(range(4), 2))
+    assert abs(best - 0.1) < 1e-12
+    kept0, _, j00 = oracle.restore_row(c, 2, rounds=0)
+    assert kept0.tolist() == [0, 1] and j00 == 2.0
+
+
+def test_restoration_without_rounds_is_top_drift_score():
+    w, q, k, v = _tiny_inputs()
+    idx, j0, j1 = oracle.select_blocks_restore(q, k, v, w.block, w.budget, rounds=0)
+    c = oracle.pooled_contributions(q, k, v, w.block)
+    score = torch.linalg.vector_norm(torch.tensor(c), dim=-1).numpy()
+    ref = np.sort(np.argsort(-score, axis=-1, kind="stable")[..., :w.budget], axis=-1)
+    assert (idx == ref).all() and np.array_equal(j0, j1)
+
+
+def test_one_round_takes_the_best_single_swap_brute_force():
+    # nb = 8, budget 4, cand = 8 covers every pair: one round must land on the
+    # best drop set one swap away from the initial set (when it beats J0).
+    w, q, k, v = _tiny_inputs()
+    c = oracle.pooled_contributions(q, k, v, w.block)
+    nb = c.shape[1]
+    for h in range(c.shape[0]):
+        for i in range(nb):
+            row = torch.tensor(c[h, i])
+            score = torch.linalg.vector_norm(row, dim=-1).numpy()
+            k0 = set(np.argsort(-score, kind="stable")[:w.budget].tolist())
+
+            def jd(kept):
+                drop = [j for j in range(nb) if j not in kept]
+                return float(torch.linalg.vector_norm(row[drop].sum(0)))
+            cands = [(jd((k0 - {a}) | {b}), b, a) for b in range(nb) if b not in k0 for a in k0]
+            jbest, b, a = min(cands)
+            kept, j0, j1 = oracle.restore_row(c[h, i], w.budget, rounds=1)
+            assert abs(j0 - jd(k0)) < 1e-13
+            if jbest < j0:
+                assert kept.tolist() == sorted((k0 - {a}) | {b}) and abs(j1 - jbest) < 1e-13
+            else:
+                assert kept.tolist() == sorted(k0) and j1 == j0
+
+
+def test_restoration_never_raises_j_and_never_beats_the_optimum():
+    w, q, k, v = _tiny_inputs()
+    c = oracle.pooled_contributions(q, k, v, w.block)
+    nb = c.shape[1]
+    idx, j0, j1 = oracle.select_blocks_restore(q, k, v, w.block, w.budget, rounds=4)
+    assert (j1 <= j0).all()
+    for h in range(c.shape[0]):
+        for i in range(nb):
+            row = torch.tensor(c[h, i])
+            opt = min(float(torch.linalg.vector_norm(row[list(set(range(nb)) - set(s))].sum(0)))
+                      for s in itertools.combinations(range(nb), w.budget))
+            assert j1[h, i] >= opt - 1e-13
+            drop = [j for j in range(nb) if j not in idx[h, i]]
+            assert abs(j1[h, i] - float(torch.linalg.vector_norm(row[drop].sum(0)))) < 1e-13
+            assert len(set(idx[h, i].tolist())) == w.budget and (np.diff(idx[h, i]) > 0).all()
+
+
+def test_restoration_stops_at_a_local_minimum():
+    # d = 1, budget 2: drift scores 1, 0, 4, 3, 0 keep {2, 3}; D = {0, 1, 4}
+    # sums to -1 (J = 1).  Every single swap gives |sum| >= 3, so restoration
+    # stops there, although the drop set {0, 2, 3} sums to 0.
+    c = np.array([[-1.0], [0.0], [4.0], [-3.0], [0.0]])
+    for s in itertools.combinations(range(5), 2):
+        if set(s) == {2, 3}:
+            continue
+        if len(set(s) & {2, 3}) == 1:          # one swap away
+            assert abs(c[list(set(range(5)) - set(s))].sum()) >= 3.0
+    kept, j0, j = oracle.restore_row(c, 2, rounds=4)
+    assert kept.tolist() == [2, 3] and j0 == 1.0 and j == 1.0
+    assert abs(c[[0, 2, 3]].sum()) == 0.0
+
+
+def test_restoration_candidates_are_the_largest_gains_and_smallest_costs():
+    # d = 1, budget 2, one candidate per side.  Scores 5, 5, 4, 3, 4, 0 keep
+    # {0, 1}; D = {2, 3, 4, 5} sums to T = 11.  Gains 2 T c_b - c_b^2 are 72,
+    # 57, 72, 0: block 2 (72, lower index than 4).  Costs 2 T c_a + c_a^2 are
+    # -85, -85: block 0.  The swap gives 11 - 4 - 5 = 2 < 11.
+    c = np.array([[-5.0], [-5.0], [4.0], [3.0], [4.0], [0.0]])
+    kept, j0, j = oracle.restore_row(c, 2, rounds=1, cand=1)
+    assert kept.tolist() == [1, 2] and j0 == 11.0 and j == 2.0
