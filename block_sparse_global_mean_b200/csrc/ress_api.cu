@@ -266,6 +266,35 @@ ress_status ress_select_blocks_cdf(const ress_shape* shape, const void* q, const
                        static_cast<cudaStream_t>(stream), &cdf);
 }
 
+size_t ress_restore_workspace_bytes(const ress_shape* shape) {
+  Geometry g;
+  if (check_shape(shape, &g) != RESS_OK) return 0;
+  return restore_layout(g).total;
+}
+
+ress_status ress_select_blocks_restore(const ress_shape* shape, const void* q, const void* k,
+                                       const void* v, int32_t budget, int32_t rounds,
+                                       int32_t candidates, int32_t* idx, float* drift_init,
+                                       float* drift_final, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  Geometry g;
+  ress_status s = check_shape(shape, &g);
+  if (s != RESS_OK) return s;
+  if ((s = check_budget(g, budget)) != RESS_OK) return s;
+  if (rounds < 0 || rounds > 64 || candidates < 1 || candidates > 16) return RESS_ERR_INVALID_ARG;
+  if (g.nb == 0) return RESS_OK;
+  if (g.nb > kMaxBlocksSelect) return RESS_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !idx || !workspace) return RESS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) || (reinterpret_cast<uintptr_t>(idx) & 3u) ||
+      (reinterpret_cast<uintptr_t>(drift_init) & 3u) ||
+      (reinterpret_cast<uintptr_t>(drift_final) & 3u))
+    return RESS_ERR_INVALID_ARG;
+  if (workspace_bytes < restore_layout(g).total) return RESS_ERR_WORKSPACE;
+  return launch_restore(g, q, k, v, budget, rounds, candidates, idx, drift_init, drift_final,
+                        static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
+}
+
 size_t ress_attn_workspace_bytes(const ress_shape* shape) {
   Geometry g;
   if (check_shape(shape, &g) != RESS_OK) return 0;

@@ -102,6 +102,19 @@ ress_status launch_attn_rows(const Geometry& g, const void* q, int64_t nq, bool 
 ress_status launch_drift(const Geometry& g, const void* q, const void* k, const void* v,
                          int budget, const int32_t* idx, const float* lse, float* drift,
                          float* set_drift, cudaStream_t st);
+// Pooling pass alone: Qbar [H][nb][64], Kbar^T and Vbar^T [H][64][nb_pad].
+ress_status launch_pool(const Geometry& g, const void* q, const void* k, const void* v,
+                        float* qbar, float* kbar_t, float* vbar_t, cudaStream_t st);
+
+// Workspace of the restoration-based selection (byte offsets).
+struct RestoreLayout {
+  size_t qbar, kbar_t, vbar_t, total;
+};
+RestoreLayout restore_layout(const Geometry& g);
+ress_status launch_restore(const Geometry& g, const void* q, const void* k, const void* v,
+                           int budget, int rounds, int cand, int32_t* idx, float* j_init,
+                           float* j_final, uint8_t* ws, cudaStream_t st);
+
 // Workspace of the special (camera, register) rows of the layout-aware
 // attention: the gathered queries [rows_pad][H][64] bf16, their outputs and
 // lse (byte offsets; total 0 when there are no special tokens).

@@ -87,6 +87,11 @@ lib.ress_block_sparse_attn_layout.argtypes = [_SHAPE, _LAYOUT, _P, _P, _P, ctype
 lib.ress_block_drift_layout.restype = ctypes.c_int
 lib.ress_block_drift_layout.argtypes = [_SHAPE, _LAYOUT, _P, _P, _P, ctypes.c_int32, _P, _P, _P,
                                         _P, _P, ctypes.c_size_t, _P]
+lib.ress_restore_workspace_bytes.restype = ctypes.c_size_t
+lib.ress_restore_workspace_bytes.argtypes = [_SHAPE]
+lib.ress_select_blocks_restore.restype = ctypes.c_int
+lib.ress_select_blocks_restore.argtypes = [_SHAPE, _P, _P, _P, ctypes.c_int32, ctypes.c_int32,
+                                           ctypes.c_int32, _P, _P, _P, _P, ctypes.c_size_t, _P]
 lib.ress_validate_idx.restype = ctypes.c_int
 lib.ress_validate_idx.argtypes = [_SHAPE, ctypes.c_int32, _P, _P]
 lib.ress_check_device_errors.restype = ctypes.c_int
@@ -438,6 +443,41 @@ def ress_block_drift_layout(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, i
                  0 if workspace is None else workspace.numel(), _stream_ptr(stream, q.device))
     _check(status, "ress_block_drift_layout")
     return drift, set_drift
+
+
+def ress_select_blocks_restore(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, budget: int,
+                               block: int, rounds: int = 4, candidates: int = 8,
+                               idx: Optional[torch.Tensor] = None,
+                               drift_init: Optional[torch.Tensor] = None,
+                               drift_final: Optional[torch.Tensor] = None,
+                               workspace: Optional[torch.Tensor] = None,
+                               stream: Optional[torch.cuda.Stream] = None
+                               ) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Stage 1 by drift with restoration: returns (idx [H, nb, budget] int32,
+    drift of the initial drop set [H, nb], drift of the result [H, nb])."""
+    _check_inputs(q, k, v)
+    sh = _shape_of(q, block)
+    n, h = q.shape[0], q.shape[1]
+    nb = n // block
+    if idx is None:
+        idx = torch.empty((h, nb, budget), dtype=torch.int32, device=q.device)
+    if drift_init is None:
+        drift_init = torch.empty((h, nb), dtype=torch.float32, device=q.device)
+    if drift_final is None:
+        drift_final = torch.empty((h, nb), dtype=torch.float32, device=q.device)
+    _check_buffer(idx, (h, nb, budget), torch.int32, q.device, "idx")
+    _check_buffer(drift_init, (h, nb), torch.float32, q.device, "drift_init")
+    _check_buffer(drift_final, (h, nb), torch.float32, q.device, "drift_final")
+    _check_workspace(workspace, q.device)
+    need = int(lib.ress_restore_workspace_bytes(ctypes.byref(sh)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    status = _on(q.device, lib.ress_select_blocks_restore, ctypes.byref(sh), _ptr(q), _ptr(k),
+                 _ptr(v), int(budget), int(rounds), int(candidates), _ptr(idx), _ptr(drift_init),
+                 _ptr(drift_final), _ptr(workspace), workspace.numel(),
+                 _stream_ptr(stream, q.device))
+    _check(status, "ress_select_blocks_restore")
+    return idx, drift_init, drift_final
 
 
 def ress_validate_idx(idx: torch.Tensor, n: int, block: int,

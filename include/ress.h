@@ -217,6 +217,41 @@ ress_status ress_select_blocks_layout(const ress_shape* shape, const ress_layout
                                       void* stream);
 
 /*
+ * Workspace bytes of ress_select_blocks_restore (0 if the shape is invalid):
+ * Qbar [H][nb][64], Kbar^T [H][64][nb_pad] and Vbar^T [H][64][nb_pad],
+ * float32, each 256-byte aligned.
+ */
+size_t ress_restore_workspace_bytes(const ress_shape* shape);
+
+/*
+ * Stage 1 by drift with iterative residual restoration (ReSS Abstract, Fig. 1,
+ * Fig. 3(b)-(c), Fig. 7, Table S3), on pooled contributions.  For query block
+ * i of head h, key block j contributes c_j = p_ij Vbar_j to the pooled output
+ * (p_ij the pooled probabilities of ress_select_blocks).  The drift score is
+ * |c_j|; the initial kept set is the `budget` blocks of largest score (ties
+ * to the lower index).  Each of up to `rounds` restoration rounds takes the
+ * drop set D and T = sum_{j in D} c_j, forms the pairs of the `candidates`
+ * dropped blocks of largest 2 <T, c_b> - |c_b|^2 and the `candidates` kept
+ * blocks of smallest 2 <T, c_a> + |c_a|^2 (ties to the lower index), and swaps
+ * the pair of smallest |T - c_b + c_a| (ties: lower b, then lower a) when
+ * that is below |T|; otherwise restoration stops.  The swap rule and the
+ * pooled contributions are this library's reading: the pages give neither.
+ *
+ *   rounds       0 .. 64 (0: the initial set).
+ *   candidates   1 .. 16 per side.
+ *   idx          out, [H][nb][budget] int32, ascending.
+ *   drift_init   out, [H][nb] float32, |sum over the initial drop set|; or NULL.
+ *   drift_final  out, [H][nb] float32, the same for the result; or NULL.
+ *   Supported sizes: nb <= 4096.  Arithmetic in float32; a decision between
+ *   two values equal to float32 rounding may go either way.
+ */
+ress_status ress_select_blocks_restore(const ress_shape* shape, const void* q, const void* k,
+                                       const void* v, int32_t budget, int32_t rounds,
+                                       int32_t candidates, int32_t* idx, float* drift_init,
+                                       float* drift_final, void* workspace,
+                                       size_t workspace_bytes, void* stream);
+
+/*
  * Workspace bytes that ress_block_sparse_attn and ress_block_drift need:
  * 0 for bf16 inputs; 3 * N * H * 64 * 2 for float32 inputs (bf16 copies of
  * q, k and v).

@@ -270,3 +270,24 @@ def test_layout_entry_points_reject_bad_layouts_on_the_host(ress):
     assert lib.ress_attn_layout_workspace_bytes(ctypes.byref(sh), ctypes.byref(none), 0) == 0
     assert lib.ress_select_blocks_layout(ctypes.byref(sh), ctypes.byref(good), FAKE, FAKE, 4,
                                          FAKE, FAKE_WS, 16, None) == ress.RESS_ERR_WORKSPACE
+
+
+@no_gpu_only
+def test_restore_rejects_bad_arguments_on_the_host(ress):
+    lib = ress.lib
+    sh = _shape(ress)                                              # nb = 8
+
+    def call(budget=4, rounds=4, cand=8, q=FAKE, v=FAKE, ws_bytes=1 << 30):
+        return lib.ress_select_blocks_restore(ctypes.byref(sh), q, FAKE, v, budget, rounds, cand,
+                                              FAKE, None, None, FAKE_WS, ws_bytes, None)
+    assert call(budget=0) == ress.RESS_ERR_INVALID_ARG
+    assert call(budget=9) == ress.RESS_ERR_INVALID_ARG
+    assert call(rounds=-1) == ress.RESS_ERR_INVALID_ARG
+    assert call(rounds=65) == ress.RESS_ERR_INVALID_ARG
+    assert call(cand=0) == ress.RESS_ERR_INVALID_ARG
+    assert call(cand=17) == ress.RESS_ERR_INVALID_ARG
+    assert call(v=None) == ress.RESS_ERR_INVALID_ARG
+    assert call(q=FAKE + 4) == ress.RESS_ERR_INVALID_ARG
+    assert call(ws_bytes=16) == ress.RESS_ERR_WORKSPACE
+    # Qbar, Kbar^T and Vbar^T (nb_pad = 256)
+    assert lib.ress_restore_workspace_bytes(ctypes.byref(sh)) == 4 * 2 * 8 * 64 + 2 * 4 * 2 * 64 * 256
