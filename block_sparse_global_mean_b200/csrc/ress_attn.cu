@@ -186,7 +186,7 @@ __device__ __forceinline__ void store_row<float>(float* dst, const float* o, flo
 
 // 10 warps: three of them share an SM sub-partition's 16,384 registers, so
 // the launch bound caps the kernel at 168 registers per thread.
-template <typename OutT>
+template <typename OutT, bool kLayout>
 __global__ void __launch_bounds__(kThreads, 1)
     block_sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
                              const __grid_constant__ CUtensorMap tm_k,
@@ -244,13 +244,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Dense pass: every key block, for both query blocks of the tile.
   for (int w = threadIdx.x; w < 2 * W; w += kThreads) {
     const int ww = w < W ? w : w - W;
-    bmA[w] = p.dense ? ((ww < p.nb >> 5) ? 0xFFFFFFFFu : ((1u << (p.nb & 31)) - 1u)) : 0u;
+    bmA[w] = (kLayout && p.dense) ? ((ww < p.nb >> 5) ? 0xFFFFFFFFu : ((1u << (p.nb & 31)) - 1u))
+                                  : 0u;
   }
   __syncthreads();
 
   // Kept sets of the tile's query blocks as bitmaps (duplicates collapse,
   // out-of-range entries are skipped and flagged).
-  for (int e = threadIdx.x; e < (p.dense ? 0 : nsets * p.budget); e += kThreads) {
+  for (int e = threadIdx.x; e < ((kLayout && p.dense) ? 0 : nsets * p.budget); e += kThreads) {
     const int s = e / p.budget;
     const int r = e - s * p.budget;
     const int qb = qb0 + s;
@@ -432,8 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t m0, m1;
       chunk_info(list, n_entries, p.block, c, t0, t1, m0, m1);
       // Valid (non-padding) prefix of each 64-key sub-block.
-      const int vk0 = layout_valid(p.lay_t, p.lay_r, t0, 64);
-      const int vk1 = layout_valid(p.lay_t, p.lay_r, t1, 64);
+      const int vk0 = kLayout ? layout_valid(p.lay_t, p.lay_r, t0, 64) : 64;
+      const int vk1 = kLayout ? layout_valid(p.lay_t, p.lay_r, t1, 64) : 64;
       const bool use0 = ((m0 >> half) & 1u) && vk0 > 0;
       const bool use1 = ((m1 >> half) & 1u) && vk1 > 0;
       if (!use0 && !use1) {
@@ -453,8 +454,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tS + 64, r[2]);
       tmem_ld32(tS + 96, r[3]);
       tmem_ld_wait();
-      if (vk0 < 64) mask_sub_block(r[0], r[1], vk0);
-      if (vk1 < 64) mask_sub_block(r[2], r[3], vk1);
+      if (kLayout) {
+        if (vk0 < 64) mask_sub_block(r[0], r[1], vk0);
+        if (vk1 < 64) mask_sub_block(r[2], r[3], vk1);
+      }
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
       if (use0) {
 #pragma unroll
@@ -537,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Epilogue: the odd-chunk group posts its row statistics; the even-chunk
     // group merges both partial results and writes the row.
     const int tok = row0 + row;
-    const bool query_pad = !p.dense && p.lay_t != 0 && (tok % p.lay_t) >= p.lay_r;
+    const bool query_pad = kLayout && !p.dense && (tok % p.lay_t) >= p.lay_r;
     if (par == 1) {
       ctl->odd_m[row] = m_ref;
       ctl->odd_lr[row] = lr_sum;
@@ -619,6 +622,18 @@ ress_status launch_exp2_poly_test(const float* x, float* y, int n, cudaStream_t 
 
 bool make_token_map(CUtensorMap* map, const void* base, const Geometry& g, int rows);
 
+template <typename OutT, bool kLayout>
+ress_status launch_attn_kernel(dim3 grid, size_t smem, const CUtensorMap& tq,
+                               const CUtensorMap& tk, const CUtensorMap& tv, const AttnParams& p,
+                               cudaStream_t st) {
+  if (ress_status s = record_cuda(cudaFuncSetAttribute(block_sparse_attn_kernel<OutT, kLayout>,
+                                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)smem)))
+    return s;
+  block_sparse_attn_kernel<OutT, kLayout><<<grid, kThreads, smem, st>>>(tq, tk, tv, p);
+  return record_cuda(cudaGetLastError());
+}
+
 ress_status launch_attn_rows(const Geometry& g, const void* q, int64_t nq, bool dense,
                              const void* k, const void* v, int budget, const int32_t* idx,
                              void* out, bool out_f32, float* lse, cudaStream_t st) {
@@ -649,18 +664,13 @@ ress_status launch_attn_rows(const Geometry& g, const void* q, int64_t nq, bool 
   const size_t smem = attn_smem_bytes(g.nb);
   if (smem > 227 * 1024) return RESS_ERR_UNSUPPORTED;   // kept-block lists no longer fit
   const dim3 grid((unsigned)(g.heads * p.tiles_per_head));
-  if (out_f32) {
-    if (ress_status st_ = record_cuda(cudaFuncSetAttribute(block_sparse_attn_kernel<float>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
-      return st_;
-    block_sparse_attn_kernel<float><<<grid, kThreads, smem, st>>>(tq, tk, tv, p);
-  } else {
-    if (ress_status st_ = record_cuda(cudaFuncSetAttribute(block_sparse_attn_kernel<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
-      return st_;
-    block_sparse_attn_kernel<__nv_bfloat16><<<grid, kThreads, smem, st>>>(tq, tk, tv, p);
-  }
-  return record_cuda(cudaGetLastError());
+  // The plain path is compiled without any of the layout's checks.
+  const bool lay = g.lay_t != 0 || dense;
+  if (out_f32)
+    return lay ? launch_attn_kernel<float, true>(grid, smem, tq, tk, tv, p, st)
+               : launch_attn_kernel<float, false>(grid, smem, tq, tk, tv, p, st);
+  return lay ? launch_attn_kernel<__nv_bfloat16, true>(grid, smem, tq, tk, tv, p, st)
+             : launch_attn_kernel<__nv_bfloat16, false>(grid, smem, tq, tk, tv, p, st);
 }
 
 ress_status launch_attn(const Geometry& g, const void* q, const void* k, const void* v,
