@@ -515,18 +515,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     named_bar_sync(1, kTcWorkers);
 
-#ifdef RESS_TC_DEBUG
-    if (live && half == 0) {
-      int32_t* o = a.idx + ((size_t)h * nb + i) * a.budget;
-      const float v[12] = {top, bot, scale, delta, hiT, loT, (float)0, (float)kept_all,
-                           (float)n0, (float)n1, (float)need, row_ok ? 1.f : 0.f};
-      for (int e = 0; e < 12 && e < a.budget; ++e) o[e] = __float_as_int(v[e]);
-    }
-    if (false) {
-#else
     // ---- write the kept blocks in ascending order, or hand the row over ----
     if (live && ok) {
-#endif
       if (row_ok) {
         int32_t* out = a.idx + ((size_t)h * nb + i) * a.budget;
         const int words = (nb + 31) >> 5;
