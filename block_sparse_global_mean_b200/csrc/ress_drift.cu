@@ -344,11 +344,14 @@ __global__ void __launch_bounds__(kThreads, B128 ? 2 : 1)
             for (int kk = 0; kk < 8; ++kk)
               mma_ts(tmem + kColC0, tS + kk * 8, dv + (uint64_t)(kk * 128), idPV, kk > 0 ? 1u : 0u);
           }
+          // The contributions are signalled as soon as they are done (a commit
+          // tracks the MMAs issued before it), so their norms overlap the
+          // running sum below and the next chunk's S.
+          mma_commit(bar_c);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             mma_ts(tmem + col_t<B128>(), tS + kk * 8, dv + (uint64_t)(kk * 128), idPV,
                    (c > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(bar_c);
           mma_commit(smem_addr(&ctl->kv_empty[s]));
           if (c == n_chunks - 1) mma_commit(bar_t);
         }

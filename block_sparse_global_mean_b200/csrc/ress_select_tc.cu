@@ -23,10 +23,10 @@
 //            score within delta of b* is a candidate, anything else is
 //            dropped.
 //
-// The candidates of a row (a few dozen at most) are then ranked exactly:
-// float32 dot products over d in ascending order, larger score first, lower
-// index first on equal scores, and the best budget - (kept outright) join the
-// row's bitmap, which is written out in ascending block order.  A row whose
+// The candidates of a row (a few dozen at most) are then ranked by their
+// full products (larger first, lower index first on equal scores), and the
+// best budget - (kept outright) join the row's bitmap, which the worker warps
+// write out in ascending block order, one row per warp at a time.  A row whose
 // band turns out not to hold the budget-th score (delta is an allowance
 // sized from the measured tf32 error, not a proof), or holds more candidates
 // than fit, is handed to the exact fallback kernel, which recomputes it.
@@ -98,6 +98,7 @@ struct __align__(8) TcCtl {
   float xb[2][kTcRows];
   int xc[2][kTcRows];
   int xd[2][kTcRows];
+  int rstate[kTcRows];   // 1: the row's bitmap is its result; 0: dead row or handed over
 };
 
 size_t tc_smem_bytes() { return 1024 + kTcStages * kTcStage + kTcRegion + sizeof(TcCtl); }
@@ -132,21 +133,19 @@ __device__ __forceinline__ void hist_pair(float s0, float s1, float2 neg_scale2,
   red_add_shared_u32(hist_row + (uint32_t)(b1 >> 1) * (kTcRows * 4), 1u + (uint32_t)(b1 & 1) * 0xFFFFu);
 }
 
-// float32 dot product of Qbar_i with key j, d in ascending order, the key read
-// back as its tf32 high + low parts (the fallback kernel's arithmetic).
-__device__ __forceinline__ float exact_score(const float* q, const float* kh, const float* kl) {
-  float acc = 0.f;
+// r[u] for a run-time u without indexing the register array (which would
+// place it in local memory): a tree of selects on the bits of u.
+__device__ __forceinline__ uint32_t select32(const uint32_t (&r)[32], int u) {
+  uint32_t l1[16], l2[8], l3[4], l4[2];
 #pragma unroll
-  for (int d4 = 0; d4 < kHeadDim / 4; ++d4) {
-    const float4 qv = *reinterpret_cast<const float4*>(q + 4 * d4);
-    const float4 hv = *reinterpret_cast<const float4*>(kh + 4 * d4);
-    const float4 lv = *reinterpret_cast<const float4*>(kl + 4 * d4);
-    acc = fmaf(qv.x, hv.x + lv.x, acc);
-    acc = fmaf(qv.y, hv.y + lv.y, acc);
-    acc = fmaf(qv.z, hv.z + lv.z, acc);
-    acc = fmaf(qv.w, hv.w + lv.w, acc);
-  }
-  return acc;
+  for (int e = 0; e < 16; ++e) l1[e] = (u & 1) ? r[2 * e + 1] : r[2 * e];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) l2[e] = (u & 2) ? l1[2 * e + 1] : l1[2 * e];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) l3[e] = (u & 4) ? l2[2 * e + 1] : l2[2 * e];
+#pragma unroll
+  for (int e = 0; e < 2; ++e) l4[e] = (u & 8) ? l3[2 * e + 1] : l3[2 * e];
+  return (u & 16) ? l4[1] : l4[0];
 }
 
 __global__ void __launch_bounds__(kTcThreads, 1)
@@ -339,11 +338,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (ok) {
         tc_fence_after();
         const uint32_t tA = tmem + kTcColAcc + lane_off + 64u * (uint32_t)half;
+        uint32_t r2[2][32];
+        tmem_ld32(tA, r2[0]);
+        tmem_ld32(tA + 32u, r2[1]);
+        tmem_ld_wait_regs(r2[0]);
+        tmem_ld_wait_regs(r2[1]);
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
-          uint32_t r[32];
-          tmem_ld32(tA + 32u * g, r);
-          tmem_ld_wait_regs(r);
+          const uint32_t (&r)[32] = r2[g];
 #pragma unroll
           for (int u = 0; u < 16; ++u) {
             const float s0 = __uint_as_float(r[2 * u]), s1 = __uint_as_float(r[2 * u + 1]);
@@ -375,11 +377,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t tA = tmem + kTcColAcc + 128u * (uint32_t)b + lane_off + 64u * (uint32_t)half;
+      uint32_t r2[2][32];
+      tmem_ld32(tA, r2[0]);
+      tmem_ld32(tA + 32u, r2[1]);
+      tmem_ld_wait_regs(r2[0]);
+      tmem_ld_wait_regs(r2[1]);
 #pragma unroll
       for (int g = 0; g < 2; ++g) {
-        uint32_t r[32];
-        tmem_ld32(tA + 32u * g, r);
-        tmem_ld_wait_regs(r);
+        const uint32_t (&r)[32] = r2[g];
         const int j0 = 128 * c + 64 * half + 32 * g;
         if (j0 + 32 <= nb) {
 #pragma unroll
@@ -442,11 +447,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t tA = tmem + kTcColAcc + 128u * (uint32_t)b + lane_off + 64u * (uint32_t)half;
+      uint32_t r2[2][32];
+      tmem_ld32(tA, r2[0]);
+      tmem_ld32(tA + 32u, r2[1]);
+      tmem_ld_wait_regs(r2[0]);
+      tmem_ld_wait_regs(r2[1]);
 #pragma unroll
       for (int g = 0; g < 2; ++g) {
-        uint32_t r[32];
-        tmem_ld32(tA + 32u * g, r);
-        tmem_ld_wait_regs(r);
+        const uint32_t (&r)[32] = r2[g];
         uint32_t kw = 0u, gw = 0u;
 #pragma unroll
         for (int u = 0; u < 32; ++u) {
@@ -466,22 +474,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         while (cw != 0u) {
           const int u = __ffs(cw) - 1;
           cw &= cw - 1u;
-          if (nc < kTcCand) cand_j[nc * kTcWorkers + wt] = (uint16_t)(j0 + u);
+          if (nc < kTcCand) {
+            cand_j[nc * kTcWorkers + wt] = (uint16_t)(j0 + u);
+            cand_s[nc * kTcWorkers + wt] = __uint_as_float(select32(r, u));
+          }
           ++nc;
         }
       }
       tc_fence_before();
       mbar_arrive(smem_addr(&ctl->acc_empty[b]));
-    }
-    // Exact scores of this thread's candidates.
-    if (ok && live) {
-      const float* kh0 = a.khi + (size_t)h * a.nb_pad * kHeadDim;
-      const float* kl0 = a.klo + (size_t)h * a.nb_pad * kHeadDim;
-      for (int n = 0; n < min(nc, kTcCand); ++n) {
-        const int j = cand_j[n * kTcWorkers + wt];
-        cand_s[n * kTcWorkers + wt] =
-            exact_score(qrow, kh0 + (size_t)j * kHeadDim, kl0 + (size_t)j * kHeadDim);
-      }
     }
     ctl->xc[half][row] = kept;
     ctl->xd[half][row] = ok ? nc : kTcCand + 1;
@@ -515,30 +516,44 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     named_bar_sync(1, kTcWorkers);
 
-    // ---- write the kept blocks in ascending order, or hand the row over ----
-    if (live && ok) {
-      if (row_ok) {
-        int32_t* out = a.idx + ((size_t)h * nb + i) * a.budget;
-        const int words = (nb + 31) >> 5;
-        int pos = 0;
-        for (int w = 0; w < words; ++w) {
-          uint32_t m = bitmap[w * kTcRows + row];
-          if (((w >> 1) & 1) == half) {
-            int p = pos;
-            while (m != 0u) {
-              const int u = __ffs(m) - 1;
-              m &= m - 1u;
-              if (p < a.budget) out[p] = 32 * w + u;
-              ++p;
-            }
-            pos = p;
-          } else {
-            pos += __popc(m);
-          }
-        }
-      } else if (half == 0) {
+    // ---- hand failed rows over; write the others in ascending order ----
+    if (half == 0) {
+      ctl->rstate[row] = (live && ok && row_ok) ? 1 : 0;
+      if (live && ok && !row_ok) {
         const int slot = atomicAdd(a.fb_count, 1);
         a.fb_list[slot] = h * nb + i;
+      }
+    }
+    named_bar_sync(1, kTcWorkers);
+    // Each worker warp writes 16 rows, a row at a time: lanes take the
+    // bitmap words, a warp prefix sum places their kept blocks, and the row's
+    // output (contiguous in idx) is written by the whole warp.
+    {
+      const int ww = wt >> 5;
+      const int words = (nb + 31) >> 5;
+      for (int rr = ww; rr < kTcRows; rr += kTcWorkers / 32) {
+        if (ctl->rstate[rr] == 0) continue;                 // warp-uniform
+        int32_t* out = a.idx + ((size_t)h * nb + i0 + rr) * a.budget;
+        int base = 0;
+        for (int w0 = 0; w0 < words; w0 += 32) {
+          const int w = w0 + lane;
+          uint32_t m = w < words ? bitmap[w * kTcRows + rr] : 0u;
+          const int cnt = __popc(m);
+          int incl = cnt;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          int at = base + incl - cnt;
+          while (m != 0u) {
+            const int u = __ffs(m) - 1;
+            m &= m - 1u;
+            if (at < a.budget) out[at] = 32 * w + u;
+            ++at;
+          }
+          base += __shfl_sync(0xffffffffu, incl, 31);
+        }
       }
     }
   }
