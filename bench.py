@@ -159,10 +159,20 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end pass")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the 200-view record (selection, attention and drift stages)")
+    ap.add_argument("--views", type=int, default=0,
+                    help="run the workload's recipe on this many views instead (small cases for "
+                         "profiler captures; not a bench configuration)")
     ap.add_argument("--shard", default="none", choices=["none", "heads"],
                     help="none: every rank runs its own input (weak scaling); heads: the ranks "
                          "split the heads of one input (strong scaling, no collective)")
     return ap.parse_args()
+
+
+def pick_workload(args):
+    w = workloads.WORKLOADS[args.workload]
+    if args.views > 0 and args.views != w.views:
+        w = workloads.scaled(w, args.views)
+    return w
 
 
 def rank_seed(w, rank: int) -> int:
@@ -268,7 +278,7 @@ def cpu_oracle_rate(w, q_cpu, k_cpu, v_cpu, seconds_target: float = 12.0, thread
 def run_reference(args, rank: int, world: int):
     if rank != 0:
         return
-    w = workloads.WORKLOADS[args.workload]
+    w = pick_workload(args)
     q, k, v = workloads.generate(w)
     rates = []
     samples = ""
@@ -457,7 +467,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = workloads.WORKLOADS[args.workload]
+    w = pick_workload(args)
     peaks, peak_kind = load_peaks()
     if args.shard == "heads":
         h0, h1 = head_slice(w.heads, world, rank)

@@ -192,8 +192,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                              const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = align1024_shared(smem_raw);
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + kQBytes;
   Ctl* ctl = reinterpret_cast<Ctl*>(sKV + kStages * kStageBytes);

@@ -57,6 +57,14 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// The first 1024-byte boundary at or after p (a dynamic shared-memory
+// array), by pointer arithmetic on the array itself: an integer round trip
+// would hide from the compiler that the result addresses shared memory, and
+// every access through it would become a generic one.
+__device__ __forceinline__ uint8_t* align1024_shared(uint8_t* p) {
+  return p + ((1024u - (static_cast<uint32_t>(__cvta_generic_to_shared(p)) & 1023u)) & 1023u);
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -85,11 +93,12 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 // Waits for the phase of `parity` to complete.  Gives up when `abort_flag`
 // (shared memory, set by any thread of the CTA) is raised or after
 // kWaitLimitNs, in which case it raises the abort flag and the device error
-// (RESS_ERR_TIMEOUT, `detail`) and returns false.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
-                                          volatile int* abort_flag, DeviceError* err,
-                                          int detail) {
-  if (mbar_try_wait(bar, parity)) return true;
+// (RESS_ERR_TIMEOUT, `detail`) and returns false.  The first probe is inline;
+// the bounded loop is an out-of-line call, so that the many wait sites of a
+// kernel do not each carry a copy of it in the instruction stream.
+static __device__ __noinline__ bool mbar_wait_slow(uint32_t bar, uint32_t parity,
+                                                   volatile int* abort_flag, DeviceError* err,
+                                                   int detail) {
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -104,11 +113,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
   }
 }
 
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity,
+                                          volatile int* abort_flag, DeviceError* err,
+                                          int detail) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, abort_flag, err, detail);
+}
+
 // Same, but ignores the abort flag (used to drain copies in flight before a
 // CTA exits).  Returns false after the time limit.
-__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, DeviceError* err,
-                                                int detail) {
-  if (mbar_try_wait(bar, parity)) return true;
+static __device__ __noinline__ bool mbar_wait_drain_slow(uint32_t bar, uint32_t parity,
+                                                         DeviceError* err, int detail) {
   const unsigned long long t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
@@ -117,6 +132,12 @@ __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, D
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, DeviceError* err,
+                                                int detail) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_drain_slow(bar, parity, err, detail);
 }
 
 // ---------------------------------------------------------------------------

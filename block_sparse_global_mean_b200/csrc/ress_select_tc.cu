@@ -7,36 +7,42 @@
 // parts; the pooled keys stream through shared memory in 128-key chunks (TMA,
 // 128-byte swizzle), also as tf32 high and low planes, and each chunk's
 // 128 x 128 scores land in one of three TMEM accumulators.  Each row is owned
-// by two worker threads (warps w and w + 4 share the TMEM lanes), one per
-// 64-column half of every chunk.  Three passes over the keys, all reading
-// the scores straight from TMEM:
+// by four worker threads (the four warps that share its TMEM lane quadrant),
+// one per 32-column quarter of every chunk.  Three passes over the keys, all
+// reading the scores straight from TMEM:
 //
 //   sample   128 evenly spaced keys, approximate scores (Qhi . Khi): the
 //            row's range [bot, top].
-//   pass A   every key, approximate scores: a histogram of 256 bins of width
-//            (top - bot) / 256 counted from the top (values outside the range
-//            fall in the end bins); bin b* holds the budget-th largest
-//            approximate score.
+//   pass A   every key, approximate scores: a histogram of 128 bins of width
+//            (top - bot) / 127 counted from the top (values outside the range
+//            saturate into the end bins); bin b* holds the budget-th largest
+//            approximate score.  The bin is formed by a saturating FMA and a
+//            round-to-integer add of 1.5 * 2^23, whose bit pattern, times the
+//            histogram's row stride, is the shared-memory address up to a
+//            constant: about 3.5 instructions per score (the saturating FMA,
+//            half a packed FMA, the address multiply-add and a shared
+//            reduction).
 //   pass B   every key, the full product Qhi.Khi + Qhi.Klo + Qlo.Khi (about
 //            float32 accuracy): a score above b*'s upper edge plus the
 //            allowance delta for the approximate pass is kept outright, a
-//            score within delta of b* is a candidate, anything else is
-//            dropped.
+//            score within delta of b* is a candidate (appended to the row's
+//            list with its full-product score), anything else is dropped.
 //
-// The candidates of a row (a few dozen at most) are then ranked by their
-// full products (larger first, lower index first on equal scores), and the
-// best budget - (kept outright) join the row's bitmap, which the worker warps
-// write out in ascending block order, one row per warp at a time.  A row whose
-// band turns out not to hold the budget-th score (delta is an allowance
-// sized from the measured tf32 error, not a proof), or holds more candidates
-// than fit, is handed to the exact fallback kernel, which recomputes it.
+// Then one warp per row: the row's candidates are ranked by their full
+// products (larger first, lower index first on equal scores), the best
+// budget - (kept outright) join the row's bitmap, and the warp unpacks the
+// bitmap in ascending block order into shared memory (sparse words by their
+// lane, dense words by the whole warp) and copies the row out coalesced.  A row whose band turns out not to hold the budget-th score (delta is
+// an allowance sized from the measured tf32 error, not a proof), or holds more
+// candidates than fit, is handed to the exact fallback kernel, which
+// recomputes it.
 //
 // Sources: ReSS (thelatestinai.com) Table S5, SpargeAttn row - selection by
 // pooled query/key inner products; Table 1 - a fused scoring kernel;
 // VASC (paperlayer.ai) A.2 - an exact-capacity binary Top-K.
 //
-// Warp roles (320 threads, one CTA per SM): warp 0 TMA, warp 1 TMEM owner and
-// MMA issuer (one elected lane), warps 2-9 workers.  Every mbarrier wait is
+// Warp roles (576 threads, one CTA per SM): warp 0 TMA, warp 1 TMEM owner and
+// MMA issuer (one elected lane), warps 2-17 workers.  Every mbarrier wait is
 // bounded; after a timeout the workers skip the remaining work but still pass
 // every named barrier, and the CTA frees TMEM and exits.
 #include "ress_common.cuh"
@@ -47,29 +53,36 @@ namespace ress {
 namespace {
 
 constexpr int kTcRows = 128;
-constexpr int kTcThreads = 320;
-constexpr int kTcWorkers = 256;
+constexpr int kTcThreads = 576;
+constexpr int kTcWorkers = 512;
 constexpr int kTcStages = 2;
 constexpr uint32_t kTcBox = 128 * 32 * 4;     // 128 keys x 32 d of float32 = one swizzle span
 constexpr uint32_t kTcPlane = 2 * kTcBox;     // 128 keys x 64 d
 constexpr uint32_t kTcStage = 2 * kTcPlane;   // tf32 high and low planes
 constexpr int kTcAcc = 3;
 constexpr uint32_t kTcColQhi = 0, kTcColQlo = 64, kTcColAcc = 128;
-constexpr int kTcCand = 32;                   // candidates per worker thread
+constexpr int kTcBins = 128;
+constexpr int kTcCand = 72;                   // candidates per row
 constexpr int kTcWords = kMaxBlocksTc / 32;   // bitmap words per row
-// Worker scratch: during pass A the row histograms, [128 words][128 rows]
-// u32 (two u16 bin counts per word); afterwards the kept-block bitmaps
-// [kTcWords][128 rows] u32, the candidate indices [kTcCand][256] u16 and
-// their exact scores [kTcCand][256] f32.
-constexpr uint32_t kTcHistBytes = 128 * kTcRows * 4;
+// Worker scratch: during pass A the row histograms, [kTcBins][128 rows] u32;
+// afterwards the kept-block bitmaps [kTcWords][128 rows] u32, the candidate
+// indices [kTcCand][128] u16 and their full-product scores [kTcCand][128] f32.
+// Bitmap words and candidate slots are stored at row ^ (word or slot & 31), so
+// that a warp touching 32 rows of one word, or 32 words of one row, hits 32
+// different banks.
+constexpr uint32_t kTcHistBytes = kTcBins * kTcRows * 4;
 constexpr uint32_t kTcBitmapBytes = kTcWords * kTcRows * 4;
-constexpr uint32_t kTcCandJBytes = kTcCand * kTcWorkers * 2;
-constexpr uint32_t kTcCandSBytes = kTcCand * kTcWorkers * 4;
+constexpr uint32_t kTcCandJBytes = kTcCand * kTcRows * 2;
+constexpr uint32_t kTcCandSBytes = kTcCand * kTcRows * 4;
 constexpr uint32_t kTcRegion = (kTcBitmapBytes + kTcCandJBytes + kTcCandSBytes) > kTcHistBytes
                                    ? (kTcBitmapBytes + kTcCandJBytes + kTcCandSBytes)
                                    : kTcHistBytes;
 constexpr uint32_t kMagicBits = 0x4B400000u;  // bits of 1.5 * 2^23
 constexpr float kMagic = 12582912.0f;
+// The bin b of a score sits in the low bits of kMagicBits + b; times the
+// histogram's row stride (512 bytes) that is b * 512 plus kMagicBits * 512,
+// which is 2^31 modulo 2^32.
+constexpr uint32_t kHistBias = kMagicBits * (uint32_t)(kTcRows * 4);
 
 struct TcArgs {
   DeviceError* err;
@@ -94,11 +107,10 @@ struct __align__(8) TcCtl {
   int abort_flag;
   uint32_t kmax_bits;
   int pad;
-  float xa[2][kTcRows];
-  float xb[2][kTcRows];
-  int xc[2][kTcRows];
-  int xd[2][kTcRows];
-  int rstate[kTcRows];   // 1: the row's bitmap is its result; 0: dead row or handed over
+  float xa[4][kTcRows];     // per quarter: the sample's largest score
+  float xb[4][kTcRows];     // per quarter: the sample's smallest score
+  int kept[kTcRows];        // scores above the band
+  int ncand[kTcRows];       // candidates appended (may exceed kTcCand)
 };
 
 size_t tc_smem_bytes() { return 1024 + kTcStages * kTcStage + kTcRegion + sizeof(TcCtl); }
@@ -118,19 +130,23 @@ __device__ __forceinline__ float to_tf32(float x) {
   return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xFFFFE000u);
 }
 
-// Histogram bin of a pair of approximate scores: t = (top - s) * scale
-// (off = top * scale), rounded to the nearest integer by adding 1.5 * 2^23
-// in a separate step (a constant that folded both would lose t's fraction to
-// the ulp of 1 at 2^23), clamped to [0, 255]; then one increment of the u16
-// count of that bin in the row's histogram.
-__device__ __forceinline__ void hist_pair(float s0, float s1, float2 neg_scale2, float2 off2,
-                                          uint32_t hist_row) {
-  const float2 t = ffma2(make_float2(s0, s1), neg_scale2, off2);
-  const float2 f = fadd2(t, make_float2(kMagic, kMagic));
-  const int b0 = min(max((int)(__float_as_uint(f.x) - kMagicBits), 0), 255);
-  const int b1 = min(max((int)(__float_as_uint(f.y) - kMagicBits), 0), 255);
-  red_add_shared_u32(hist_row + (uint32_t)(b0 >> 1) * (kTcRows * 4), 1u + (uint32_t)(b0 & 1) * 0xFFFFu);
-  red_add_shared_u32(hist_row + (uint32_t)(b1 >> 1) * (kTcRows * 4), 1u + (uint32_t)(b1 & 1) * 0xFFFFu);
+// min(max(a * b + c, 0), 1) in one instruction.
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Histogram count of a pair of approximate scores: u = sat((top - s) / (top -
+// bot)) (NaN saturates to 0), b = round(127 u) by adding 1.5 * 2^23 (so the
+// float's bits are kMagicBits + b), and one increment of the row's bin b at
+// hist_row + 512 b = hist_row - kHistBias + 512 * bits (modulo 2^32).
+__device__ __forceinline__ void hist_pair(float s0, float s1, float neg_us, float off,
+                                          uint32_t hist_base) {
+  const float2 f = ffma2(make_float2(fma_sat(s0, neg_us, off), fma_sat(s1, neg_us, off)),
+                         make_float2(127.0f, 127.0f), make_float2(kMagic, kMagic));
+  red_add_shared_u32(hist_base + __float_as_uint(f.x) * (uint32_t)(kTcRows * 4), 1u);
+  red_add_shared_u32(hist_base + __float_as_uint(f.y) * (uint32_t)(kTcRows * 4), 1u);
 }
 
 // r[u] for a run-time u without indexing the register array (which would
@@ -148,13 +164,16 @@ __device__ __forceinline__ uint32_t select32(const uint32_t (&r)[32], int u) {
   return (u & 16) ? l4[1] : l4[0];
 }
 
+__device__ __forceinline__ uint32_t swz(int word_or_slot, int row) {
+  return (uint32_t)(word_or_slot * kTcRows + (row ^ (word_or_slot & 31)));
+}
+
 __global__ void __launch_bounds__(kTcThreads, 1)
     topk_tc_kernel(const __grid_constant__ CUtensorMap tm_khi,
                    const __grid_constant__ CUtensorMap tm_klo,
                    const __grid_constant__ CUtensorMap tm_ks, const TcArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  uint8_t* smem = align1024_shared(smem_raw);
   uint8_t* stages = smem;
   uint8_t* region = smem + kTcStages * kTcStage;
   TcCtl* ctl = reinterpret_cast<TcCtl*>(region + kTcRegion);
@@ -277,40 +296,54 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     __syncwarp();
   } else {
     // ---------------- workers ----------------
-    const int wt = threadIdx.x - 64;            // 0 .. 255
+    const int wt = threadIdx.x - 64;            // 0 .. 511
     const int quad = warp & 3;                  // TMEM lanes 32 quad .. 32 quad + 31
-    const int half = (warp - 2) >> 2;           // columns 64 half .. 64 half + 63 of a chunk
+    const int quarter = (warp - 2) >> 2;        // columns 32 quarter .. 32 quarter + 31 of a chunk
     const int row = quad * 32 + lane;
     const int i = i0 + row;
     const bool live = i < a.nb;
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t col = 32u * (uint32_t)quarter;
     const int nb = a.nb;
     const float* qrow = a.qbar + ((size_t)h * nb + (live ? i : 0)) * kHeadDim;
     bool ok = true;
 
-    // Zero the histograms (64 KB over the 256 workers).
+    // Zero the histograms (64 KB over the 512 workers) and the row counters.
     {
       uint4* z = reinterpret_cast<uint4*>(region);
       for (int e = wt; e < (int)(kTcHistBytes / 16); e += kTcWorkers) z[e] = make_uint4(0u, 0u, 0u, 0u);
+      if (quarter == 0) {
+        ctl->kept[row] = 0;
+        ctl->ncand[row] = 0;
+      }
     }
-    // Qbar row into TMEM: half 0 writes the tf32 high parts, half 1 the low.
+    // Qbar row into TMEM: quarter q writes d = 32 (q & 1) .. + 31 of the tf32
+    // high (q < 2) or low (q >= 2) parts.  Every thread sums |Qbar_i|^2.
     float qn2 = 0.f;
-#pragma unroll
-    for (int g = 0; g < 2; ++g) {
+    {
+      const float* qown = qrow + 32 * (quarter & 1);
       uint32_t part[32];
 #pragma unroll
       for (int u4 = 0; u4 < 8; ++u4) {
-        float4 x = live ? *reinterpret_cast<const float4*>(qrow + 32 * g + 4 * u4)
-                        : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 x = live ? *reinterpret_cast<const float4*>(qown + 4 * u4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
         const float xs[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float hi = to_tf32(xs[e]);
-          part[4 * u4 + e] = __float_as_uint(half ? to_tf32(xs[e] - hi) : hi);
           qn2 = fmaf(xs[e], xs[e], qn2);
+          const float hi = to_tf32(xs[e]);
+          part[4 * u4 + e] = __float_as_uint(quarter >= 2 ? to_tf32(xs[e] - hi) : hi);
         }
       }
-      tmem_st32(tmem + (half ? kTcColQlo : kTcColQhi) + lane_off + 32u * (uint32_t)g, part);
+      tmem_st32(tmem + (quarter >= 2 ? kTcColQlo : kTcColQhi) + lane_off + 32u * (uint32_t)(quarter & 1),
+                part);
+      const float* qother = qrow + 32 * ((quarter & 1) ^ 1);
+#pragma unroll 1
+      for (int u4 = 0; u4 < 8; ++u4) {
+        const float4 x = live ? *reinterpret_cast<const float4*>(qother + 4 * u4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+        qn2 = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, fmaf(x.w, x.w, qn2))));
+      }
     }
     // Largest key norm of the head.
     {
@@ -331,229 +364,250 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const float delta = sqrtf(qn2) * kmax * (1.0f / 2048.0f);
 
     // ---- sample: the row's range ----
-    float top = 0.f, bot = 0.f;
     {
       float mx = -INFINITY, mn = INFINITY;
       if (ok) ok = warp_wait(smem_addr(&ctl->acc_full[0]), 0, abortf, a.err, 96);
       if (ok) {
         tc_fence_after();
-        const uint32_t tA = tmem + kTcColAcc + lane_off + 64u * (uint32_t)half;
-        uint32_t r2[2][32];
-        tmem_ld32(tA, r2[0]);
-        tmem_ld32(tA + 32u, r2[1]);
-        tmem_ld_wait_regs(r2[0]);
-        tmem_ld_wait_regs(r2[1]);
+        uint32_t r[32];
+        tmem_ld32(tmem + kTcColAcc + lane_off + col, r);
+        tmem_ld_wait_regs(r);
 #pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          const uint32_t (&r)[32] = r2[g];
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const float s0 = __uint_as_float(r[2 * u]), s1 = __uint_as_float(r[2 * u + 1]);
-            mx = fmax3(mx, s0, s1);
-            mn = fminf(mn, fminf(s0, s1));
-          }
+        for (int u = 0; u < 16; ++u) {
+          const float s0 = __uint_as_float(r[2 * u]), s1 = __uint_as_float(r[2 * u + 1]);
+          mx = fmax3(mx, s0, s1);
+          mn = fminf(mn, fminf(s0, s1));
         }
         tc_fence_before();
         mbar_arrive(smem_addr(&ctl->acc_empty[0]));
       }
-      ctl->xa[half][row] = mx;
-      ctl->xb[half][row] = mn;
+      ctl->xa[quarter][row] = mx;
+      ctl->xb[quarter][row] = mn;
     }
     named_bar_sync(1, kTcWorkers);
-    top = fmaxf(ctl->xa[0][row], ctl->xa[1][row]);
-    bot = fminf(ctl->xb[0][row], ctl->xb[1][row]);
-    float scale = 256.0f / (top - bot);
+    const float top = fmaxf(fmaxf(ctl->xa[0][row], ctl->xa[1][row]),
+                            fmaxf(ctl->xa[2][row], ctl->xa[3][row]));
+    const float bot = fminf(fminf(ctl->xb[0][row], ctl->xb[1][row]),
+                            fminf(ctl->xb[2][row], ctl->xb[3][row]));
+    // t = (top - s) * scale in [0, 127] across the sample's range.
+    float scale = (float)(kTcBins - 1) / (top - bot);
     if (!(scale < INFINITY)) scale = 0.f;           // constant range: one bin
-    const float2 neg_scale2 = make_float2(-scale, -scale);
-    const float off = top * scale;
-    const float2 off2 = make_float2(off, off);
+    const float us = 1.0f / (top - bot) < INFINITY ? 1.0f / (top - bot) : 0.f;
+    const float neg_us = -us, off = top * us;
 
     // ---- pass A: histogram of the approximate scores ----
-    const uint32_t hist_row = smem_addr(region) + (uint32_t)row * 4u;
-    for (int c = 0; c < C && ok; ++c) {
-      const int seq = 1 + c;
+    // Every column is counted, the last chunk's padding too: TMA fills the
+    // key rows past nb with zeros, whose score is exactly 0, so the scan
+    // below takes their count (pad) back out of the bin that 0 falls in.
+    const uint32_t hist_base = smem_addr(region) + (uint32_t)row * 4u - kHistBias;
+    auto load_chunk = [&](int seq, uint32_t (&r)[32], int detail) -> bool {
       const int b = seq % kTcAcc;
-      ok = warp_wait(smem_addr(&ctl->acc_full[b]), (seq / kTcAcc) & 1, abortf, a.err, 97);
-      if (!ok) break;
+      if (!warp_wait(smem_addr(&ctl->acc_full[b]), (seq / kTcAcc) & 1, abortf, a.err, detail))
+        return false;
       tc_fence_after();
-      const uint32_t tA = tmem + kTcColAcc + 128u * (uint32_t)b + lane_off + 64u * (uint32_t)half;
-      uint32_t r2[2][32];
-      tmem_ld32(tA, r2[0]);
-      tmem_ld32(tA + 32u, r2[1]);
-      tmem_ld_wait_regs(r2[0]);
-      tmem_ld_wait_regs(r2[1]);
-#pragma unroll
-      for (int g = 0; g < 2; ++g) {
-        const uint32_t (&r)[32] = r2[g];
-        const int j0 = 128 * c + 64 * half + 32 * g;
-        if (j0 + 32 <= nb) {
-#pragma unroll
-          for (int u = 0; u < 16; ++u)
-            hist_pair(__uint_as_float(r[2 * u]), __uint_as_float(r[2 * u + 1]), neg_scale2, off2,
-                      hist_row);
-        } else {
-#pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            if (j0 + u < nb) {
-              const float t = fmaf(__uint_as_float(r[u]), neg_scale2.x, off2.x);
-              const int b0 = min(max((int)(__float_as_uint(t + kMagic) - kMagicBits), 0), 255);
-              red_add_shared_u32(hist_row + (uint32_t)(b0 >> 1) * (kTcRows * 4),
-                                 1u + (uint32_t)(b0 & 1) * 0xFFFFu);
-            }
-          }
-        }
-      }
+      tmem_ld32(tmem + kTcColAcc + 128u * (uint32_t)b + lane_off + col, r);
+      tmem_ld_wait_regs(r);
       tc_fence_before();
       mbar_arrive(smem_addr(&ctl->acc_empty[b]));
+      return true;
+    };
+    for (int c = 0; c < C && ok; ++c) {
+      uint32_t r[32];
+      ok = load_chunk(1 + c, r, 97);
+      if (!ok) break;
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        hist_pair(__uint_as_float(r[2 * u]), __uint_as_float(r[2 * u + 1]), neg_us, off, hist_base);
     }
     named_bar_sync(1, kTcWorkers);
 
     // ---- the bin b* of the budget-th largest approximate score ----
-    // Both threads of a row scan the same counts, so they agree without an
-    // exchange.  Bin 0 is the top of the range.
+    // The four threads of a row scan the same counts, so they agree without
+    // an exchange.  Bin 0 is the top of the range.
     float hiT = INFINITY, loT = -INFINITY;
     {
       const uint32_t* hist = reinterpret_cast<const uint32_t*>(region);
-      int cum = 0, bstar = 255;
-      for (int w = 0; w < 128; ++w) {
-        const uint32_t v = hist[w * kTcRows + row];
-        const int c0 = (int)(v & 0xFFFFu), c1 = (int)(v >> 16);
-        if (cum + c0 >= a.budget) { bstar = 2 * w; break; }
-        cum += c0;
-        if (cum + c1 >= a.budget) { bstar = 2 * w + 1; break; }
-        cum += c1;
+      const int pad = 128 * C - nb;
+      const int bin0 = (int)(__float_as_uint(fmaf(fma_sat(0.0f, neg_us, off), 127.0f, kMagic)) -
+                             kMagicBits);
+      int cum = 0, bstar = kTcBins - 1;
+      for (int b0 = 0; b0 < kTcBins; b0 += 8) {
+        int v[8], s8 = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          v[e] = (int)hist[(b0 + e) * kTcRows + row] - (b0 + e == bin0 ? pad : 0);
+          s8 += v[e];
+        }
+        if (cum + s8 >= a.budget) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            if (cum + v[e] >= a.budget) {
+              bstar = b0 + e;
+              break;
+            }
+            cum += v[e];
+          }
+          break;
+        }
+        cum += s8;
       }
       // Bin b holds the approximate scores s with (top - s) * scale within
-      // 1/2 of b (bin 0 everything above, bin 255 everything below the
+      // 1/2 of b (bin 0 everything above, the last bin everything below the
       // range), up to rounding; the exact budget-th score lies within delta
       // of b*.
       const float eps = 1e-6f * (fabsf(top) + fabsf(bot)) + 1e-30f;
       if (scale > 0.f) {
         if (bstar > 0) hiT = top - ((float)bstar - 0.5f) / scale + delta + eps;
-        if (bstar < 255) loT = top - ((float)bstar + 0.5f) / scale - delta - eps;
+        if (bstar < kTcBins - 1) loT = top - ((float)bstar + 0.5f) / scale - delta - eps;
       }
     }
     named_bar_sync(1, kTcWorkers);   // the histograms are no longer read
 
     // ---- pass B: full products; keep, candidate or drop ----
     uint32_t* bitmap = reinterpret_cast<uint32_t*>(region);                           // [words][128]
-    uint16_t* cand_j = reinterpret_cast<uint16_t*>(region + kTcBitmapBytes);          // [cap][256]
-    float* cand_s = reinterpret_cast<float*>(region + kTcBitmapBytes + kTcCandJBytes); // [cap][256]
-    int kept = 0, nc = 0;
+    uint16_t* cand_j = reinterpret_cast<uint16_t*>(region + kTcBitmapBytes);          // [cap][128]
+    float* cand_s = reinterpret_cast<float*>(region + kTcBitmapBytes + kTcCandJBytes); // [cap][128]
+    int kept = 0;
     for (int c = 0; c < C && ok; ++c) {
-      const int seq = C + 1 + c;
-      const int b = seq % kTcAcc;
-      ok = warp_wait(smem_addr(&ctl->acc_full[b]), (seq / kTcAcc) & 1, abortf, a.err, 98);
+      uint32_t r[32];
+      ok = load_chunk(C + 1 + c, r, 98);
       if (!ok) break;
-      tc_fence_after();
-      const uint32_t tA = tmem + kTcColAcc + 128u * (uint32_t)b + lane_off + 64u * (uint32_t)half;
-      uint32_t r2[2][32];
-      tmem_ld32(tA, r2[0]);
-      tmem_ld32(tA + 32u, r2[1]);
-      tmem_ld_wait_regs(r2[0]);
-      tmem_ld_wait_regs(r2[1]);
+      uint32_t kw = 0u, gw = 0u;
 #pragma unroll
-      for (int g = 0; g < 2; ++g) {
-        const uint32_t (&r)[32] = r2[g];
-        uint32_t kw = 0u, gw = 0u;
-#pragma unroll
-        for (int u = 0; u < 32; ++u) {
-          const float sv = __uint_as_float(r[u]);
-          kw |= (sv > hiT) ? (1u << u) : 0u;
-          gw |= (sv >= loT) ? (1u << u) : 0u;
-        }
-        const int j0 = 128 * c + 64 * half + 32 * g;
-        if (j0 + 32 > nb) {
-          const uint32_t valid = j0 >= nb ? 0u : ((1u << (nb - j0)) - 1u);
-          kw &= valid;
-          gw &= valid;
-        }
-        if (j0 < nb) bitmap[(j0 >> 5) * kTcRows + row] = kw;
-        kept += __popc(kw);
-        uint32_t cw = gw & ~kw;
-        while (cw != 0u) {
-          const int u = __ffs(cw) - 1;
-          cw &= cw - 1u;
-          if (nc < kTcCand) {
-            cand_j[nc * kTcWorkers + wt] = (uint16_t)(j0 + u);
-            cand_s[nc * kTcWorkers + wt] = __uint_as_float(select32(r, u));
-          }
-          ++nc;
+      for (int u = 0; u < 32; ++u) {
+        const float sv = __uint_as_float(r[u]);
+        kw |= (sv > hiT) ? (1u << u) : 0u;
+        gw |= (sv >= loT) ? (1u << u) : 0u;
+      }
+      const int j0 = 128 * c + (int)col;
+      if (j0 + 32 > nb) {
+        const uint32_t valid = j0 >= nb ? 0u : ((1u << (nb - j0)) - 1u);
+        kw &= valid;
+        gw &= valid;
+      }
+      if (j0 < nb) bitmap[swz(j0 >> 5, row)] = kw;
+      kept += __popc(kw);
+      uint32_t cw = gw & ~kw;
+      while (cw != 0u) {
+        const int u = __ffs(cw) - 1;
+        cw &= cw - 1u;
+        const int slot = atomicAdd(&ctl->ncand[row], 1);
+        if (slot < kTcCand) {
+          cand_j[swz(slot, row)] = (uint16_t)(j0 + u);
+          cand_s[swz(slot, row)] = __uint_as_float(select32(r, u));
         }
       }
-      tc_fence_before();
-      mbar_arrive(smem_addr(&ctl->acc_empty[b]));
     }
-    ctl->xc[half][row] = kept;
-    ctl->xd[half][row] = ok ? nc : kTcCand + 1;
+    if (kept > 0) atomicAdd(&ctl->kept[row], kept);
     named_bar_sync(1, kTcWorkers);
 
-    // ---- rank the candidates; winners join the bitmap ----
-    const int kept_all = ctl->xc[0][row] + ctl->xc[1][row];
-    const int n0 = ctl->xd[0][row], n1 = ctl->xd[1][row];
-    const int need = a.budget - kept_all;
-    const bool row_ok = ok && n0 <= kTcCand && n1 <= kTcCand && need >= 0 && need <= n0 + n1;
-    if (row_ok && live && need > 0) {
-      const int wt_other = wt ^ 128;               // the row's other thread
-      const int n_other = half ? n0 : n1;
-      for (int n = 0; n < nc; ++n) {
-        const int jx = cand_j[n * kTcWorkers + wt];
-        const float sx = cand_s[n * kTcWorkers + wt];
+    // ---- one warp per row: rank the candidates, then write the row ----
+    const bool aborted = *abortf != 0;
+    const int ww = wt >> 5;
+    const int words = (nb + 31) >> 5;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    // Output staging of this warp (the key stages are free once pass B is
+    // done): 1,024 entries per warp, a row segment at a time.
+    constexpr int kSeg = 1024;
+    int32_t* stg = reinterpret_cast<int32_t*>(stages) + ww * kSeg;
+    for (int rr = ww; rr < kTcRows; rr += kTcWorkers / 32) {
+      if (aborted || i0 + rr >= nb) break;
+      const int total = ctl->ncand[rr];
+      const int need = a.budget - ctl->kept[rr];
+      if (!(total <= kTcCand && need >= 0 && need <= total)) {
+        if (lane == 0) {
+          const int slot = atomicAdd(a.fb_count, 1);
+          a.fb_list[slot] = h * nb + i0 + rr;
+        }
+        continue;
+      }
+      // Rank: the number of candidates with a larger full-product score, or
+      // an equal score and a lower block index; the best `need` win.
+      if (need > 0 && total <= 32) {
+        const float sx = lane < total ? cand_s[swz(lane, rr)] : -INFINITY;
+        const int jx = lane < total ? (int)cand_j[swz(lane, rr)] : 0xFFFF;
         int rank = 0;
-        for (int m = 0; m < nc; ++m) {
-          const float sy = cand_s[m * kTcWorkers + wt];
-          const int jy = cand_j[m * kTcWorkers + wt];
+#pragma unroll 4
+        for (int m = 0; m < total; ++m) {
+          const float sy = __shfl_sync(0xffffffffu, sx, m);
+          const int jy = __shfl_sync(0xffffffffu, jx, m);
           rank += (sy > sx || (sy == sx && jy < jx)) ? 1 : 0;
         }
-        for (int m = 0; m < n_other; ++m) {
-          const float sy = cand_s[m * kTcWorkers + wt_other];
-          const int jy = cand_j[m * kTcWorkers + wt_other];
-          rank += (sy > sx || (sy == sx && jy < jx)) ? 1 : 0;
-        }
-        // The word of block jx belongs to this thread's half of the chunk.
-        if (rank < need) bitmap[(jx >> 5) * kTcRows + row] |= 1u << (jx & 31);
-      }
-    }
-    named_bar_sync(1, kTcWorkers);
-
-    // ---- hand failed rows over; write the others in ascending order ----
-    if (half == 0) {
-      ctl->rstate[row] = (live && ok && row_ok) ? 1 : 0;
-      if (live && ok && !row_ok) {
-        const int slot = atomicAdd(a.fb_count, 1);
-        a.fb_list[slot] = h * nb + i;
-      }
-    }
-    named_bar_sync(1, kTcWorkers);
-    // Each worker warp writes 16 rows, a row at a time: lanes take the
-    // bitmap words, a warp prefix sum places their kept blocks, and the row's
-    // output (contiguous in idx) is written by the whole warp.
-    {
-      const int ww = wt >> 5;
-      const int words = (nb + 31) >> 5;
-      for (int rr = ww; rr < kTcRows; rr += kTcWorkers / 32) {
-        if (ctl->rstate[rr] == 0) continue;                 // warp-uniform
-        int32_t* out = a.idx + ((size_t)h * nb + i0 + rr) * a.budget;
-        int base = 0;
-        for (int w0 = 0; w0 < words; w0 += 32) {
-          const int w = w0 + lane;
-          uint32_t m = w < words ? bitmap[w * kTcRows + rr] : 0u;
-          const int cnt = __popc(m);
-          int incl = cnt;
+        if (lane < total && rank < need) atomicOr(&bitmap[swz(jx >> 5, rr)], 1u << (jx & 31));
+      } else if (need > 0) {
+        float sx[3];
+        int jx[3], rank[3] = {0, 0, 0};
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += y;
-          }
-          int at = base + incl - cnt;
-          while (m != 0u) {
-            const int u = __ffs(m) - 1;
-            m &= m - 1u;
-            if (at < a.budget) out[at] = 32 * w + u;
-            ++at;
-          }
-          base += __shfl_sync(0xffffffffu, incl, 31);
+        for (int t = 0; t < 3; ++t) {
+          const int cx = 32 * t + lane;
+          sx[t] = cx < total ? cand_s[swz(cx, rr)] : -INFINITY;
+          jx[t] = cx < total ? (int)cand_j[swz(cx, rr)] : 0xFFFF;
         }
+#pragma unroll 2
+        for (int m = 0; m < total; ++m) {
+          const float sy = cand_s[swz(m, rr)];
+          const int jy = cand_j[swz(m, rr)];
+#pragma unroll
+          for (int t = 0; t < 3; ++t)
+            rank[t] += (sy > sx[t] || (sy == sx[t] && jy < jx[t])) ? 1 : 0;
+        }
+#pragma unroll
+        for (int t = 0; t < 3; ++t)
+          if (32 * t + lane < total && rank[t] < need)
+            atomicOr(&bitmap[swz(jx[t] >> 5, rr)], 1u << (jx[t] & 31));
+      }
+      __syncwarp();
+      // Write: lane l holds bitmap words l, l + 32 and l + 64; a warp scan
+      // gives every word's first output position.  Words with at most 8
+      // blocks are unpacked by their lane; denser words (whole views kept)
+      // by the whole warp, one word at a time.  Both go through the staging
+      // buffer, which the warp then copies out in 128-byte rows.
+      uint32_t mw[3];
+      int base[3], run = 0;
+#pragma unroll
+      for (int t = 0; t < 3; ++t) {
+        const int w = 32 * t + lane;
+        mw[t] = w < words ? bitmap[swz(w, rr)] : 0u;
+        const int c = __popc(mw[t]);
+        int incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        base[t] = run + incl - c;
+        run += __shfl_sync(0xffffffffu, incl, 31);
+      }
+      const int n_out = min(run, a.budget);
+      int32_t* out = a.idx + ((size_t)h * nb + i0 + rr) * a.budget;
+      for (int s0 = 0; s0 < n_out; s0 += kSeg) {
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+          const int wbase = 32 * (32 * t + lane);
+          if (__popc(mw[t]) <= 8) {
+            uint32_t m = mw[t];
+            int pos = base[t] - s0;
+            while (m != 0u) {
+              const int u = __ffs(m) - 1;
+              m &= m - 1u;
+              if (pos >= 0 && pos < kSeg) stg[pos] = wbase + u;
+              ++pos;
+            }
+          }
+          uint32_t dense = __ballot_sync(0xffffffffu, __popc(mw[t]) > 8);
+          while (dense != 0u) {
+            const int src = __ffs(dense) - 1;
+            dense &= dense - 1u;
+            const uint32_t word = __shfl_sync(0xffffffffu, mw[t], src);
+            const int pos = __shfl_sync(0xffffffffu, base[t], src) + __popc(word & lt_mask) - s0;
+            if (((word >> lane) & 1u) && pos >= 0 && pos < kSeg)
+              stg[pos] = 32 * (32 * t + src) + lane;
+          }
+        }
+        __syncwarp();
+        const int n_seg = min(n_out - s0, kSeg);
+        for (int e = lane; e < n_seg; e += 32) out[s0 + e] = stg[e];
+        __syncwarp();
       }
     }
   }
