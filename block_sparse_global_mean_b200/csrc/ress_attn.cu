@@ -24,7 +24,10 @@
 //              with a lazy rescale of O (only when the running maximum grows
 //              by more than 2^8), and P goes back to TMEM as bf16 over the
 //              first 64 columns of S; epilogue O / sum(P) and lse, where
-//              sum(P) adds the same bf16-rounded values that enter P V.
+//              sum(P) adds the same bf16-rounded values that enter P V (so
+//              that the rounding of a dominant probability cancels in O).
+//              Three exponentials in four go to MUFU and one to a
+//              polynomial on the FMA pipe.
 //
 // Every mbarrier wait is bounded; on timeout the CTA raises the device error,
 // drains its copies and MMAs in flight, frees TMEM and exits.
@@ -457,22 +460,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (vk0 < 64) mask_sub_block(r[0], r[1], vk0);
         if (vk1 < 64) mask_sub_block(r[2], r[3], vk1);
       }
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+      // Chunk maximum over eight independent chains (short dependency).
+      float mxa[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) mxa[q] = -INFINITY;
       if (use0) {
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          mx0 = fmax3(mx0, __uint_as_float(r[0][2 * u]), __uint_as_float(r[0][2 * u + 1]));
-          mx1 = fmax3(mx1, __uint_as_float(r[1][2 * u]), __uint_as_float(r[1][2 * u + 1]));
+        for (int u = 0; u < 8; ++u) {
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            mxa[2 * g] = fmax3(mxa[2 * g], __uint_as_float(r[g][4 * u]), __uint_as_float(r[g][4 * u + 1]));
+            mxa[2 * g + 1] =
+                fmax3(mxa[2 * g + 1], __uint_as_float(r[g][4 * u + 2]), __uint_as_float(r[g][4 * u + 3]));
+          }
         }
       }
       if (use1) {
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          mx2 = fmax3(mx2, __uint_as_float(r[2][2 * u]), __uint_as_float(r[2][2 * u + 1]));
-          mx3 = fmax3(mx3, __uint_as_float(r[3][2 * u]), __uint_as_float(r[3][2 * u + 1]));
+        for (int u = 0; u < 8; ++u) {
+#pragma unroll
+          for (int g = 2; g < 4; ++g) {
+            mxa[2 * g] = fmax3(mxa[2 * g], __uint_as_float(r[g][4 * u]), __uint_as_float(r[g][4 * u + 1]));
+            mxa[2 * g + 1] =
+                fmax3(mxa[2 * g + 1], __uint_as_float(r[g][4 * u + 2]), __uint_as_float(r[g][4 * u + 3]));
+          }
         }
       }
-      const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      const float mx = fmaxf(fmaxf(fmax3(mxa[0], mxa[1], mxa[2]), fmax3(mxa[3], mxa[4], mxa[5])),
+                             fmaxf(mxa[6], mxa[7]));
       // Lazy rescale: a row moves its reference maximum only when the chunk's
       // maximum exceeds it by more than 8 (a factor 2^8 in p); O and its row
       // sums are rescaled after P is written (below).
@@ -496,8 +511,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 16; ++e) {
             const float2 sv = make_float2(__uint_as_float(r[g][2 * e]), __uint_as_float(r[g][2 * e + 1]));
             const float2 x = ffma2(sv, scale2, neg_m2);
-            // One pair in eight goes to the FMA pipe, the rest to MUFU.
-            const float2 pe = ((e & 7) == 7) ? exp2_poly2(x)
+            // One pair in four goes to the FMA pipe, the rest to MUFU.
+            const float2 pe = ((e & 3) == 3) ? exp2_poly2(x)
                                              : make_float2(fast_exp2(x.x), fast_exp2(x.y));
             pk[e] = pack_bf16x2(pe.x, pe.y);
             lr_lo = add_bf16_lo(pk[e], lr_lo);

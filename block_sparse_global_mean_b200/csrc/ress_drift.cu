@@ -376,6 +376,8 @@ __global__ void __launch_bounds__(kThreads, B128 ? 2 : 1)
     const float lse2 =
         (tok < p.n && live_q) ? p.lse[(size_t)h * p.n + tok] * 1.4426950408889634f : 0.f;
     const float neg_l = -lse2;
+    const float2 neg_l2 = make_float2(neg_l, neg_l);
+    const float2 scale2 = make_float2(kScaleLog2, kScaleLog2);
     const int sub_tid = threadIdx.x - 64;   // 0..127 among the softmax warps
     bool ok = true;
     for (int c = 0; c < n_chunks; ++c) {
@@ -403,11 +405,14 @@ __global__ void __launch_bounds__(kThreads, B128 ? 2 : 1)
             uint32_t pk[16];
             const int vk = hf == 0 ? vk0 : vk1;
             if (use && vk == 64 && all_live) {
+              // One pair in four on the FMA pipe (polynomial), the rest on MUFU.
 #pragma unroll
               for (int e = 0; e < 16; ++e) {
-                const float p0 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e]), kScaleLog2, neg_l));
-                const float p1 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e + 1]), kScaleLog2, neg_l));
-                pk[e] = pack_bf16x2(p0, p1);
+                const float2 x = ffma2(make_float2(__uint_as_float(r[g][2 * e]), __uint_as_float(r[g][2 * e + 1])),
+                                       scale2, neg_l2);
+                const float2 pe = ((e & 3) == 3) ? exp2_poly2(x)
+                                                 : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+                pk[e] = pack_bf16x2(pe.x, pe.y);
               }
             } else {
               // Layout: padding keys (columns beyond the sub-block's valid
@@ -440,29 +445,29 @@ __global__ void __launch_bounds__(kThreads, B128 ? 2 : 1)
       tc_fence_after();
       float ss0 = 0.f, ss1 = 0.f;
       {
-        uint32_t cv[32];
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          tmem_ld32(tmem + kColC0 + lane_off + 32 * g, cv);
+        // Sum of squares over the 64 columns of a contribution: packed pairs
+        // into four independent accumulators (a short dependency chain).
+        auto sumsq64 = [&](uint32_t col) -> float {
+          uint32_t cv[2][32];
+          tmem_ld32(tmem + col + lane_off, cv[0]);
+          tmem_ld32(tmem + col + lane_off + 32, cv[1]);
           tmem_ld_wait();
+          float2 acc[4];
 #pragma unroll
-          for (int u = 0; u < 32; ++u) {
-            const float x = __uint_as_float(cv[u]);
-            ss0 = fmaf(x, x, ss0);
-          }
-        }
-        if (p.block == 64) {
+          for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
 #pragma unroll
           for (int g = 0; g < 2; ++g) {
-            tmem_ld32(tmem + kColC1 + lane_off + 32 * g, cv);
-            tmem_ld_wait();
 #pragma unroll
-            for (int u = 0; u < 32; ++u) {
-              const float x = __uint_as_float(cv[u]);
-              ss1 = fmaf(x, x, ss1);
+            for (int u = 0; u < 16; ++u) {
+              const float2 x = make_float2(__uint_as_float(cv[g][2 * u]), __uint_as_float(cv[g][2 * u + 1]));
+              acc[u & 3] = ffma2(x, x, acc[u & 3]);
             }
           }
-        }
+          return ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                 ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+        };
+        ss0 = sumsq64(kColC0);
+        if (p.block == 64) ss1 = sumsq64(kColC1);
       }
       tc_fence_before();
       mbar_arrive(bar_cf);
