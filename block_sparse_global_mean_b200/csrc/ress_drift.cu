@@ -17,12 +17,12 @@
 // measures that shift per block, and the drift of a drop set depends on the
 // directions of the contributions, so the set drift is the norm of their sum.
 //
-// Warp roles as in the attention kernel (warp 0 TMA, warp 1 TMEM + MMA,
-// warps 2-5 exponentials and reductions).  Each CTA runs the chunk chain
-// S -> P -> C_j -> ||C_j|| serially; with 128-token blocks a CTA needs 256
-// TMEM columns (S, C, T) and two CTAs share an SM, so that one CTA's
-// exponentials overlap the other's MMAs and reductions.  With 64-token blocks
-// (two contributions per chunk) a CTA takes all 512 columns.
+// Two kernels share this design.  With 64-token blocks (two contributions per
+// chunk, all 512 TMEM columns) block_drift_kernel runs the chunk chain
+// S -> P -> C_j -> ||C_j|| serially with warps 0 TMA, 1 TMEM + MMA and 2-5
+// exponentials and reductions.  With 128-token blocks drift128_kernel (below)
+// splits the chunks over two softmax groups, so that one group's exponentials
+// overlap the other's contribution MMA and reduction.
 #include "ress_common.cuh"
 #include "ress_internal.h"
 
@@ -39,10 +39,7 @@ constexpr uint32_t kStageBytes = 4 * kSubBytes;
 constexpr uint32_t kColS = 0;     // S (fp32) / P (bf16, cols 0..63)
 constexpr uint32_t kColC0 = 128;  // contribution of sub-block 0 (or the whole 128-key block)
 constexpr uint32_t kColC1 = 192;  // contribution of sub-block 1 (block 64 only)
-// TMEM columns and the running sum's column: 256 / 192 for 128-token blocks
-// (C1 unused), 512 / 256 for 64-token blocks.
-template <bool B128> constexpr uint32_t tmem_cols() { return B128 ? 256u : 512u; }
-template <bool B128> constexpr uint32_t col_t() { return B128 ? 192u : 256u; }
+constexpr uint32_t kColT = 256;   // running sum T (block_drift_kernel)
 constexpr size_t kOneCtaSmem = 116 * 1024;
 
 struct DriftParams {
@@ -132,8 +129,7 @@ __device__ __forceinline__ int dropped_rank(const uint32_t* kept, const uint32_t
   return j - (int)(prefix[j >> 5] + __popc(below));
 }
 
-template <bool B128>
-__global__ void __launch_bounds__(kThreads, B128 ? 2 : 1)
+__global__ void __launch_bounds__(kThreads, 1)
     block_drift_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v, const DriftParams p) {
@@ -188,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, B128 ? 2 : 1)
     fence_mbarrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(&ctl->tmem_base), tmem_cols<B128>());
+    tmem_alloc(smem_addr(&ctl->tmem_base), 512);
     tmem_relinquish();
   }
   for (int w = threadIdx.x; w < 2 * W; w += kThreads) keptA[w] = 0u;
@@ -349,7 +345,7 @@ __global__ void __launch_bounds__(kThreads, B128 ? 2 : 1)
           mma_commit(bar_c);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + col_t<B128>(), tS + kk * 8, dv + (uint64_t)(kk * 128), idPV,
+            mma_ts(tmem + kColT, tS + kk * 8, dv + (uint64_t)(kk * 128), idPV,
                    (c > 0 || kk > 0) ? 1u : 0u);
           mma_commit(smem_addr(&ctl->kv_empty[s]));
           if (c == n_chunks - 1) mma_commit(bar_t);
@@ -521,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, B128 ? 2 : 1)
         uint32_t tv[32];
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
-          tmem_ld32(tmem + col_t<B128>() + lane_off + 32 * g, tv);
+          tmem_ld32(tmem + kColT + lane_off + 32 * g, tv);
           tmem_ld_wait();
 #pragma unroll
           for (int u = 0; u < 32; ++u) {
@@ -555,7 +551,409 @@ __global__ void __launch_bounds__(kThreads, B128 ? 2 : 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, tmem_cols<B128>());
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// 128-token blocks: one CTA per SM, two softmax groups on alternate chunks.
+//
+// The chunk chain S -> P -> C -> ||C|| of one 128-row tile is split over two
+// groups of four softmax warps (warps 2-5 the even chunks, warps 6-9 the odd
+// ones), each with its own S buffer (P written over its first 64 columns) and
+// its own contribution accumulator in TMEM; the running sum T is shared and
+// accumulated by the tensor core for both.  While one group waits for its
+// contribution's MMA and reduces it, the other computes exponentials.
+// TMEM: S0 0..127, S1 128..255, C0 256..319, C1 320..383, T 384..447.
+// ---------------------------------------------------------------------------
+constexpr int kThreads2 = 320;
+constexpr int kStages2 = 4;
+constexpr uint32_t kColC2 = 256, kColT2 = 384;
+
+struct __align__(8) Ctl2 {
+  uint64_t q_full;
+  uint64_t kv_full[kStages2];
+  uint64_t kv_empty[kStages2];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t c_full[2];
+  uint64_t c_free[2];
+  uint64_t red_full[2];
+  uint64_t t_full;
+  uint64_t tred_full;
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+  int n_entries;
+  int pad;
+  float partial[2][2][4];   // [group][chunk parity][quad]
+  float tpartial[4];
+};
+
+size_t drift128_smem_bytes(int nb) {
+  return 1024 + kQBytes + kStages2 * kStageBytes + sizeof(Ctl2) +
+         sizeof(uint32_t) * (2 * (size_t)words_for(nb) + (size_t)nb);
+}
+
+__global__ void __launch_bounds__(kThreads2, 1)
+    drift128_kernel(const __grid_constant__ CUtensorMap tm_q,
+                    const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const DriftParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024_shared(smem_raw);
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + kQBytes;
+  Ctl2* ctl = reinterpret_cast<Ctl2*>(sKV + kStages2 * kStageBytes);
+  const int W = words_for(p.nb);
+  uint32_t* kept = reinterpret_cast<uint32_t*>(ctl + 1);
+  uint32_t* pref = kept + W;
+  uint32_t* list = pref + W;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int h = blockIdx.x / p.tiles_per_head;
+  const int qb = blockIdx.x % p.tiles_per_head;
+  const int row0 = qb * kRows;
+  const int n_drop = p.nb - p.budget;
+
+  const uint32_t bar_q = smem_addr(&ctl->q_full);
+  const uint32_t bar_s0 = smem_addr(&ctl->s_full[0]);
+  const uint32_t bar_p0 = smem_addr(&ctl->p_full[0]);
+  const uint32_t bar_c0 = smem_addr(&ctl->c_full[0]);
+  const uint32_t bar_cf0 = smem_addr(&ctl->c_free[0]);
+  const uint32_t bar_r0 = smem_addr(&ctl->red_full[0]);
+  const uint32_t bar_t = smem_addr(&ctl->t_full);
+  const uint32_t bar_tred = smem_addr(&ctl->tred_full);
+  const uint32_t bar_done = smem_addr(&ctl->mma_done);
+  volatile int* abortf = &ctl->abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < kStages2; ++s) {
+      mbar_init(smem_addr(&ctl->kv_full[s]), 1);
+      mbar_init(smem_addr(&ctl->kv_empty[s]), 1);
+    }
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(bar_s0 + 8 * g, 1);
+      mbar_init(bar_p0 + 8 * g, 128);
+      mbar_init(bar_c0 + 8 * g, 1);
+      mbar_init(bar_cf0 + 8 * g, 128);
+      mbar_init(bar_r0 + 8 * g, 128);
+    }
+    mbar_init(bar_t, 1);
+    mbar_init(bar_tred, 128);
+    mbar_init(bar_done, 1);
+    ctl->abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(&ctl->tmem_base), 512);
+    tmem_relinquish();
+  }
+  for (int w = threadIdx.x; w < W; w += kThreads2) kept[w] = 0u;
+  __syncthreads();
+
+  for (int r = threadIdx.x; r < p.budget; r += kThreads2) {
+    const int j = p.idx[((size_t)h * p.nb + qb) * p.budget + r];
+    if (j < 0 || j >= p.nb) {
+      raise_device_error(p.err, RESS_ERR_BAD_INDEX, 2);
+      continue;
+    }
+    // A block named twice leaves more than nb - budget blocks dropped.
+    if (atomicOr(&kept[j >> 5], 1u << (j & 31)) & (1u << (j & 31)))
+      raise_device_error(p.err, RESS_ERR_BAD_INDEX, 5);
+  }
+  __syncthreads();
+
+  // Prefix popcounts of the kept bitmap and the list of dropped blocks.
+  if (warp == 0) {
+    int base = 0, basek = 0;
+    for (int w0 = 0; w0 < W; w0 += 32) {
+      const int w = w0 + lane;
+      uint32_t valid = 0u;
+      if (w < W) valid = (w == W - 1 && (p.nb & 31)) ? ((1u << (p.nb & 31)) - 1u) : 0xffffffffu;
+      const uint32_t k = (w < W) ? kept[w] : 0u;
+      uint32_t u = ~k & valid;
+      const int ck = __popc(k), cu = __popc(u);
+      int ik = ck, iu = cu;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int yk = __shfl_up_sync(0xffffffffu, ik, o);
+        const int yu = __shfl_up_sync(0xffffffffu, iu, o);
+        if (lane >= o) {
+          ik += yk;
+          iu += yu;
+        }
+      }
+      if (w < W) pref[w] = (uint32_t)(basek + ik - ck);
+      basek += __shfl_sync(0xffffffffu, ik, 31);
+      int pos = base + iu - cu;
+      while (u) {
+        const int bit = __ffs(u) - 1;
+        u &= u - 1u;
+        list[pos++] = (uint32_t)(w * 32 + bit);
+      }
+      base += __shfl_sync(0xffffffffu, iu, 31);
+    }
+    if (lane == 0) ctl->n_entries = base;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const uint32_t tmem = ctl->tmem_base;
+  const int n_chunks = ctl->n_entries;
+
+  if (warp == 0) {
+    // TMA producer: K and V of one dropped 128-token block per stage.
+    if (n_chunks > 0) {
+      if (elect_one()) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        mbar_arrive_expect_tx(bar_q, kQBytes);
+        tma_load_3d(smem_addr(sQ), &tm_q, bar_q, 0, h, row0);
+      }
+      __syncwarp();
+      int issued = 0;
+      for (int c = 0; c < n_chunks; ++c) {
+        const int s = c % kStages2;
+        if (c >= kStages2 &&
+            !warp_wait(smem_addr(&ctl->kv_empty[s]), ((c / kStages2) - 1) & 1, abortf, p.err, 40))
+          break;
+        const int t0 = (int)list[c] * 128;
+        const uint32_t st = smem_addr(sKV) + (uint32_t)s * kStageBytes;
+        const uint32_t bar = smem_addr(&ctl->kv_full[s]);
+        if (elect_one()) {
+          mbar_arrive_expect_tx(bar, kStageBytes);
+          tma_load_3d(st, &tm_k, bar, 0, h, t0);
+          tma_load_3d(st + kSubBytes, &tm_k, bar, 0, h, t0 + 64);
+          tma_load_3d(st + 2 * kSubBytes, &tm_v, bar, 0, h, t0);
+          tma_load_3d(st + 3 * kSubBytes, &tm_v, bar, 0, h, t0 + 64);
+        }
+        __syncwarp();
+        issued = c + 1;
+      }
+      for (int c = issued > kStages2 ? issued - kStages2 : 0; c < issued; ++c)
+        mbar_wait_drain(smem_addr(&ctl->kv_full[c % kStages2]), (c / kStages2) & 1, p.err, 41);
+      mbar_wait_drain(bar_q, 0, p.err, 42);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // MMA issuer.  Per chunk c of group g = c & 1: C(c) into C_g once P(c) is
+    // written and C(c - 2) has been read, T += P(c) V(c), then S(c + 2) into
+    // S_g (the tensor core runs the MMAs in issue order, so C(c) and T have
+    // read P(c) before S(c + 2) overwrites it).
+    if (n_chunks > 0) {
+      constexpr uint32_t idS = idesc_bf16_f32(128, 128, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(128, 64, true);
+      const uint64_t dq = smem_desc_sw128(smem_addr(sQ), 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(smem_addr(sKV), 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(smem_addr(sKV) + 2 * kSubBytes, 16384, 1024);
+      constexpr uint64_t kStageDesc = kStageBytes >> 4;
+      bool ok = warp_wait(bar_q, 0, abortf, p.err, 50);
+      auto issue_s = [&](int c) -> bool {
+        const int s = c % kStages2;
+        if (!warp_wait(smem_addr(&ctl->kv_full[s]), (c / kStages2) & 1, abortf, p.err, 51))
+          return false;
+        tc_fence_after();
+        const uint64_t dk = dk0 + (uint64_t)s * kStageDesc;
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + 128u * (uint32_t)(c & 1), dq + (uint64_t)(kk * 2), dk + (uint64_t)(kk * 2),
+                   idS, kk > 0 ? 1u : 0u);
+          mma_commit(bar_s0 + 8u * (uint32_t)(c & 1));
+        }
+        __syncwarp();
+        return true;
+      };
+      for (int c = 0; ok && c < n_chunks && c < 2; ++c) ok = issue_s(c);
+      for (int c = 0; ok && c < n_chunks; ++c) {
+        const int g = c & 1, it = c >> 1;
+        if (!warp_wait(bar_p0 + 8u * (uint32_t)g, (uint32_t)it & 1u, abortf, p.err, 52)) break;
+        if (it > 0 && !warp_wait(bar_cf0 + 8u * (uint32_t)g, (uint32_t)(it - 1) & 1u, abortf, p.err, 53))
+          break;
+        tc_fence_after();
+        const int s = c % kStages2;
+        const uint64_t dv = dv0 + (uint64_t)s * kStageDesc;
+        const uint32_t tP = tmem + 128u * (uint32_t)g;
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + kColC2 + 64u * (uint32_t)g, tP + kk * 8, dv + (uint64_t)(kk * 128), idPV,
+                   kk > 0 ? 1u : 0u);
+          mma_commit(bar_c0 + 8u * (uint32_t)g);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts(tmem + kColT2, tP + kk * 8, dv + (uint64_t)(kk * 128), idPV,
+                   (c > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(smem_addr(&ctl->kv_empty[s]));
+          if (c == n_chunks - 1) mma_commit(bar_t);
+        }
+        __syncwarp();
+        if (c + 2 < n_chunks && !(ok = issue_s(c + 2))) break;
+      }
+      if (elect_one()) mma_commit(bar_done);
+      __syncwarp();
+      mbar_wait_drain(bar_done, 0, p.err, 54);
+    }
+    __syncwarp();
+  } else {
+    const int quad = warp & 3;
+    const int grp = (warp - 2) >> 2;
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + 128u * (uint32_t)grp + lane_off;
+    const uint32_t tC = tmem + kColC2 + 64u * (uint32_t)grp + lane_off;
+    const uint32_t bar_s = bar_s0 + 8u * (uint32_t)grp;
+    const uint32_t bar_p = bar_p0 + 8u * (uint32_t)grp;
+    const uint32_t bar_c = bar_c0 + 8u * (uint32_t)grp;
+    const uint32_t bar_cf = bar_cf0 + 8u * (uint32_t)grp;
+    const uint32_t bar_red = bar_r0 + 8u * (uint32_t)grp;
+    const float kScaleLog2 = 1.4426950408889634f * 0.125f;
+    const int tok = row0 + row;
+    // Layout: only the valid, non-special queries drop anything.
+    const int pos = p.lay_t != 0 ? tok % p.lay_t : 0;
+    const bool live_q = p.lay_t == 0 || (pos < p.lay_r && pos >= p.lay_s);
+    const bool all_live = __all_sync(0xffffffffu, live_q);
+    const float lse2 =
+        (tok < p.n && live_q) ? p.lse[(size_t)h * p.n + tok] * 1.4426950408889634f : 0.f;
+    const float2 neg_l2 = make_float2(-lse2, -lse2);
+    const float2 scale2 = make_float2(kScaleLog2, kScaleLog2);
+    const int gtid = threadIdx.x - 64 - 128 * grp;   // 0..127 within the group
+    bool ok = true;
+    for (int c = grp, it = 0; c < n_chunks; c += 2, ++it) {
+      const uint32_t ph = (uint32_t)it & 1u;
+      if (!warp_wait(bar_s, ph, abortf, p.err, 60)) { ok = false; break; }
+      tc_fence_after();
+      const int j = (int)list[c];
+      const int t0 = j * 128;
+      // Two halves of 64 columns; P (bf16, two per column) of half hf goes
+      // to columns 32 hf .. 32 hf + 31, below the S columns still unread.
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const int vk = layout_valid(p.lay_t, p.lay_r, t0 + 64 * hf, 64);
+        uint32_t r[2][32];
+        tmem_ld32(tS + 64 * hf, r[0]);
+        tmem_ld32(tS + 64 * hf + 32, r[1]);
+        tmem_ld_wait();
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          uint32_t pk[16];
+          if (vk == 64 && all_live) {
+            // One pair in four on the FMA pipe (polynomial), the rest on MUFU.
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float2 x = ffma2(make_float2(__uint_as_float(r[g][2 * e]), __uint_as_float(r[g][2 * e + 1])),
+                                     scale2, neg_l2);
+              const float2 pe = ((e & 3) == 3) ? exp2_poly2(x)
+                                               : make_float2(fast_exp2(x.x), fast_exp2(x.y));
+              pk[e] = pack_bf16x2(pe.x, pe.y);
+            }
+          } else {
+            // Layout: padding keys (columns beyond the sub-block's valid
+            // prefix) and the rows of padding and special queries add nothing.
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int col = 32 * g + 2 * e;
+              float p0 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e]), kScaleLog2, neg_l2.x));
+              float p1 = fast_exp2(fmaf(__uint_as_float(r[g][2 * e + 1]), kScaleLog2, neg_l2.x));
+              if (!live_q || col >= vk) p0 = 0.f;
+              if (!live_q || col + 1 >= vk) p1 = 0.f;
+              pk[e] = pack_bf16x2(p0, p1);
+            }
+          }
+          tmem_st16(tS + 32 * hf + 16 * g, pk);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(bar_p);
+
+      if (!warp_wait(bar_c, ph, abortf, p.err, 61)) { ok = false; break; }
+      tc_fence_after();
+      float ss;
+      {
+        // Sum of squares of the row's 64 contribution columns: packed pairs
+        // into four independent accumulators.
+        uint32_t cv[2][32];
+        tmem_ld32(tC, cv[0]);
+        tmem_ld32(tC + 32, cv[1]);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(bar_cf);
+        float2 acc[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const float2 x = make_float2(__uint_as_float(cv[g][2 * u]), __uint_as_float(cv[g][2 * u + 1]));
+            acc[u & 3] = ffma2(x, x, acc[u & 3]);
+          }
+        }
+        ss = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+             ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+      }
+      ss = warp_sum(ss);
+      if (lane == 0) ctl->partial[grp][ph][quad] = ss;
+      __syncwarp();
+      mbar_arrive(bar_red);
+      // One writer per group.  A slot is rewritten two of the group's chunks
+      // later at the earliest, and no warp of the group runs that far ahead
+      // of the writer (each chunk's C waits for all 128 threads of the group).
+      if (gtid == 0 && mbar_wait(bar_red, ph, abortf, p.err, 63)) {
+        const float tot = ctl->partial[grp][ph][0] + ctl->partial[grp][ph][1] +
+                          ctl->partial[grp][ph][2] + ctl->partial[grp][ph][3];
+        const int rnk = dropped_rank(kept, pref, j);
+        if (rnk >= 0 && rnk < n_drop)
+          p.drift[((size_t)h * p.nb + qb) * n_drop + rnk] = sqrtf(tot);
+        else
+          raise_device_error(p.err, RESS_ERR_BAD_INDEX, 3);
+      }
+      __syncwarp();
+    }
+    // Drop-set drift J = ||sum_j C_j||_F (group 0).
+    if (grp == 0) {
+      float tss = 0.f;
+      if (ok && n_chunks > 0 && warp_wait(bar_t, 0, abortf, p.err, 62)) {
+        tc_fence_after();
+        uint32_t tv[2][32];
+        tmem_ld32(tmem + kColT2 + lane_off, tv[0]);
+        tmem_ld32(tmem + kColT2 + lane_off + 32, tv[1]);
+        tmem_ld_wait();
+        float2 acc[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+#pragma unroll
+          for (int u = 0; u < 16; ++u) {
+            const float2 x = make_float2(__uint_as_float(tv[g][2 * u]), __uint_as_float(tv[g][2 * u + 1]));
+            acc[u & 3] = ffma2(x, x, acc[u & 3]);
+          }
+        }
+        tss = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+              ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+      }
+      tss = warp_sum(tss);
+      if (lane == 0) ctl->tpartial[quad] = tss;
+      __syncwarp();
+      mbar_arrive(bar_tred);
+      if (p.set_drift && gtid == 0 && mbar_wait(bar_tred, 0, abortf, p.err, 64))
+        p.set_drift[(size_t)h * p.nb + qb] = sqrtf(ctl->tpartial[0] + ctl->tpartial[1] +
+                                                   ctl->tpartial[2] + ctl->tpartial[3]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -588,18 +986,20 @@ ress_status launch_drift(const Geometry& g, const void* q, const void* k, const 
   if (smem > 227 * 1024) return RESS_ERR_UNSUPPORTED;   // block lists no longer fit
   const unsigned grid = (unsigned)(g.heads * p.tiles_per_head);
   if (g.block == 128) {
+    const size_t smem2 = drift128_smem_bytes(g.nb);
+    if (smem2 > 227 * 1024) return RESS_ERR_UNSUPPORTED;
     if (ress_status st_ = record_cuda(cudaFuncSetAttribute(
-            block_drift_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+            drift128_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem2)))
       return st_;
-    block_drift_kernel<true><<<grid, kThreads, smem, st>>>(tq, tk, tv, p);
+    drift128_kernel<<<grid, kThreads2, smem2, st>>>(tq, tk, tv, p);
   } else {
     // All 512 TMEM columns per CTA: at least 116 KB of shared memory keeps a
     // second CTA (which would only wait in its TMEM allocation) off the SM.
     const size_t smem1 = smem > kOneCtaSmem ? smem : kOneCtaSmem;
     if (ress_status st_ = record_cuda(cudaFuncSetAttribute(
-            block_drift_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)))
+            block_drift_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1)))
       return st_;
-    block_drift_kernel<false><<<grid, kThreads, smem1, st>>>(tq, tk, tv, p);
+    block_drift_kernel<<<grid, kThreads, smem1, st>>>(tq, tk, tv, p);
   }
   return record_cuda(cudaGetLastError());
 }
