@@ -562,14 +562,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 // The chunk chain S -> P -> C -> ||C|| of one 128-row tile is split over two
 // groups of four softmax warps (warps 2-5 the even chunks, warps 6-9 the odd
 // ones), each with its own S buffer (P written over its first 64 columns) and
-// its own contribution accumulator in TMEM; the running sum T is shared and
-// accumulated by the tensor core for both.  While one group waits for its
-// contribution's MMA and reduces it, the other computes exponentials.
-// TMEM: S0 0..127, S1 128..255, C0 256..319, C1 320..383, T 384..447.
+// its own contribution accumulator in TMEM.  While one group waits for its
+// contribution's MMA and reduces it, the other computes exponentials.  The
+// running sum T is the sum of the contributions the softmax threads read
+// anyway: each thread adds its row of every C_j into registers, and the two
+// groups' partial sums meet in shared memory at the end (no running-sum MMA).
+// TMEM: S0 0..127, S1 128..255, C0 256..319, C1 320..383.
 // ---------------------------------------------------------------------------
 constexpr int kThreads2 = 320;
 constexpr int kStages2 = 4;
-constexpr uint32_t kColC2 = 256, kColT2 = 384;
+constexpr uint32_t kColC2 = 256;
+constexpr int kTStride = 68;   // floats per row of the shared running-sum exchange (padded)
 
 struct __align__(8) Ctl2 {
   uint64_t q_full;
@@ -580,7 +583,7 @@ struct __align__(8) Ctl2 {
   uint64_t c_full[2];
   uint64_t c_free[2];
   uint64_t red_full[2];
-  uint64_t t_full;
+  uint64_t t_post;      // group 1 wrote its running sums
   uint64_t tred_full;
   uint64_t mma_done;
   uint32_t tmem_base;
@@ -592,7 +595,7 @@ struct __align__(8) Ctl2 {
 };
 
 size_t drift128_smem_bytes(int nb) {
-  return 1024 + kQBytes + kStages2 * kStageBytes + sizeof(Ctl2) +
+  return 1024 + kQBytes + kStages2 * kStageBytes + sizeof(float) * kRows * kTStride + sizeof(Ctl2) +
          sizeof(uint32_t) * (2 * (size_t)words_for(nb) + (size_t)nb);
 }
 
@@ -604,7 +607,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
   uint8_t* smem = align1024_shared(smem_raw);
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + kQBytes;
-  Ctl2* ctl = reinterpret_cast<Ctl2*>(sKV + kStages2 * kStageBytes);
+  float* sT = reinterpret_cast<float*>(sKV + kStages2 * kStageBytes);   // [128][kTStride]
+  Ctl2* ctl = reinterpret_cast<Ctl2*>(sT + kRows * kTStride);
   const int W = words_for(p.nb);
   uint32_t* kept = reinterpret_cast<uint32_t*>(ctl + 1);
   uint32_t* pref = kept + W;
@@ -623,7 +627,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
   const uint32_t bar_c0 = smem_addr(&ctl->c_full[0]);
   const uint32_t bar_cf0 = smem_addr(&ctl->c_free[0]);
   const uint32_t bar_r0 = smem_addr(&ctl->red_full[0]);
-  const uint32_t bar_t = smem_addr(&ctl->t_full);
+  const uint32_t bar_tp = smem_addr(&ctl->t_post);
   const uint32_t bar_tred = smem_addr(&ctl->tred_full);
   const uint32_t bar_done = smem_addr(&ctl->mma_done);
   volatile int* abortf = &ctl->abort_flag;
@@ -641,7 +645,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
       mbar_init(bar_cf0 + 8 * g, 128);
       mbar_init(bar_r0 + 8 * g, 128);
     }
-    mbar_init(bar_t, 1);
+    mbar_init(bar_tp, 128);
     mbar_init(bar_tred, 128);
     mbar_init(bar_done, 1);
     ctl->abort_flag = 0;
@@ -742,9 +746,9 @@ __global__ void __launch_bounds__(kThreads2, 1)
     __syncwarp();
   } else if (warp == 1) {
     // MMA issuer.  Per chunk c of group g = c & 1: C(c) into C_g once P(c) is
-    // written and C(c - 2) has been read, T += P(c) V(c), then S(c + 2) into
-    // S_g (the tensor core runs the MMAs in issue order, so C(c) and T have
-    // read P(c) before S(c + 2) overwrites it).
+    // written and C(c - 2) has been read, then S(c + 2) into S_g (the tensor
+    // core runs the MMAs in issue order, so C(c) has read P(c) before
+    // S(c + 2) overwrites it).
     if (n_chunks > 0) {
       constexpr uint32_t idS = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idPV = idesc_bf16_f32(128, 64, true);
@@ -785,12 +789,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
             mma_ts(tmem + kColC2 + 64u * (uint32_t)g, tP + kk * 8, dv + (uint64_t)(kk * 128), idPV,
                    kk > 0 ? 1u : 0u);
           mma_commit(bar_c0 + 8u * (uint32_t)g);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts(tmem + kColT2, tP + kk * 8, dv + (uint64_t)(kk * 128), idPV,
-                   (c > 0 || kk > 0) ? 1u : 0u);
           mma_commit(smem_addr(&ctl->kv_empty[s]));
-          if (c == n_chunks - 1) mma_commit(bar_t);
         }
         __syncwarp();
         if (c + 2 < n_chunks && !(ok = issue_s(c + 2))) break;
@@ -824,6 +823,9 @@ __global__ void __launch_bounds__(kThreads2, 1)
     const float2 scale2 = make_float2(kScaleLog2, kScaleLog2);
     const int gtid = threadIdx.x - 64 - 128 * grp;   // 0..127 within the group
     bool ok = true;
+    float2 tsum[32];   // this row's share of T = sum of the group's contributions
+#pragma unroll
+    for (int u = 0; u < 32; ++u) tsum[u] = make_float2(0.f, 0.f);
     for (int c = grp, it = 0; c < n_chunks; c += 2, ++it) {
       const uint32_t ph = (uint32_t)it & 1u;
       if (!warp_wait(bar_s, ph, abortf, p.err, 60)) { ok = false; break; }
@@ -893,6 +895,7 @@ __global__ void __launch_bounds__(kThreads2, 1)
           for (int u = 0; u < 16; ++u) {
             const float2 x = make_float2(__uint_as_float(cv[g][2 * u]), __uint_as_float(cv[g][2 * u + 1]));
             acc[u & 3] = ffma2(x, x, acc[u & 3]);
+            tsum[16 * g + u] = fadd2(tsum[16 * g + u], x);
           }
         }
         ss = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
@@ -916,25 +919,28 @@ __global__ void __launch_bounds__(kThreads2, 1)
       }
       __syncwarp();
     }
-    // Drop-set drift J = ||sum_j C_j||_F (group 0).
-    if (grp == 0) {
+    // Drop-set drift J = ||sum_j C_j||_F: group 1 posts its running sums,
+    // group 0 adds its own and reduces.
+    float* trow = sT + row * kTStride;
+    if (grp == 1) {
+#pragma unroll
+      for (int u = 0; u < 16; ++u)
+        *reinterpret_cast<float4*>(trow + 4 * u) =
+            make_float4(tsum[2 * u].x, tsum[2 * u].y, tsum[2 * u + 1].x, tsum[2 * u + 1].y);
+      mbar_arrive(bar_tp);
+    } else {
       float tss = 0.f;
-      if (ok && n_chunks > 0 && warp_wait(bar_t, 0, abortf, p.err, 62)) {
-        tc_fence_after();
-        uint32_t tv[2][32];
-        tmem_ld32(tmem + kColT2 + lane_off, tv[0]);
-        tmem_ld32(tmem + kColT2 + lane_off + 32, tv[1]);
-        tmem_ld_wait();
+      if (mbar_wait(bar_tp, 0, abortf, p.err, 62)) {
         float2 acc[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int g = 0; g < 2; ++g) {
-#pragma unroll
-          for (int u = 0; u < 16; ++u) {
-            const float2 x = make_float2(__uint_as_float(tv[g][2 * u]), __uint_as_float(tv[g][2 * u + 1]));
-            acc[u & 3] = ffma2(x, x, acc[u & 3]);
-          }
+        for (int u = 0; u < 16; ++u) {
+          const float4 o = *reinterpret_cast<const float4*>(trow + 4 * u);
+          const float2 a = fadd2(tsum[2 * u], make_float2(o.x, o.y));
+          const float2 b = fadd2(tsum[2 * u + 1], make_float2(o.z, o.w));
+          acc[u & 3] = ffma2(a, a, acc[u & 3]);
+          acc[u & 3] = ffma2(b, b, acc[u & 3]);
         }
         tss = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
               ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
