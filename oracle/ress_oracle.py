@@ -562,3 +562,156 @@ def select_blocks_restore(q, k, v, block: int, budget: int, rounds: int, cand: i
         for i in range(nb):
             idx[h, i], j_init[h, i], j_final[h, i] = restore_row(contrib[h, i], budget, rounds, cand)
     return idx, j_init, j_final
+
+
+# ---------------------------------------------------------------------------
+# VASC: value-aware demand, budgeted binary execution, cross-layer memory
+# ---------------------------------------------------------------------------
+
+def block_pairs(nb: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Fixed pairs of adjacent key blocks in native order.
+
+    VASC A.1: neighbouring children in native order form fixed pairs, and an
+    unpaired final child is a singleton.  Returns (pair_of [nb]: the pair of
+    each block, size [n_pairs]: 2, or 1 for a final singleton).
+    """
+    pair_of = np.arange(nb) // 2
+    n_pairs = (nb + 1) // 2
+    size = np.full(n_pairs, 2, dtype=np.int64)
+    if nb % 2 == 1:
+        size[-1] = 1
+    return pair_of, size
+
+
+def pair_contrast(vbar) -> np.ndarray:
+    """rho[h, p]: the RMS contrast of the pooled values of pair p.
+
+    VASC 4.1 and A.3: the two children of a pair share one contrast signal,
+    the root mean square over the head dimension of the difference of their
+    pooled values; a singleton is paired with itself, so its contrast is 0.
+        rho[h, p] = sqrt( (1/d) * sum_d (Vbar[h, 2p, d] - Vbar[h, 2p+1, d])^2 )
+    """
+    vbar = _f64(vbar)
+    h, nb, d = vbar.shape
+    n_pairs = (nb + 1) // 2
+    rho = np.zeros((h, n_pairs), dtype=np.float64)
+    for p in range(nb // 2):
+        diff = vbar[:, 2 * p, :] - vbar[:, 2 * p + 1, :]
+        rho[:, p] = np.sqrt((diff * diff).sum(axis=-1) / d)
+    return rho
+
+
+def vasc_demand(probs, rho, budgets, value_aware: bool = True) -> np.ndarray:
+    """Current demand a[h, i, j] of every (head, query block, key block).
+
+    VASC 4.1: the pair's contrast modulates the query's relevance, and the
+    demand is rescaled and clipped to the query's capacity; A.2: every entry
+    is at most one and the row's total at most the capacity.  Readings:
+      * relevance is the pooled probability p_ij, modulated by multiplying
+        with the contrast of j's pair (with value_aware False the contrast
+        is one: the ablation that sets the paired-value contrast to one,
+        VASC Appendix D);
+      * the rescaling is proportional to the row's capacity c_h (ReSS Fig. 3
+        and Table 2 give each head its own budget c_h) and the clip is
+        applied once:
+            d_ij = p_ij * rho[h, pair(j)]
+            a_ij = min(1, c_h * d_ij / sum_j d_ij)   (0 when the sum is 0).
+    """
+    p = _f64(probs)
+    h_count, nbq, nb = p.shape
+    pair_of, _ = block_pairs(nb)
+    if value_aware:
+        factor = _f64(rho)[:, pair_of]                    # [H, nb]
+    else:
+        factor = np.ones((h_count, nb), dtype=np.float64)
+    a = np.zeros_like(p)
+    for h in range(h_count):
+        c = float(budgets[h])
+        for i in range(nbq):
+            d = p[h, i] * factor[h]
+            total = d.sum()
+            if total > 0.0:
+                a[h, i] = np.minimum(1.0, c * d / total)
+    return a
+
+
+def memory_ranking_copy(memory) -> np.ndarray:
+    """The copy of the pair memory that enters the ranking.
+
+    VASC A.4: normalisation runs per batch entry and head and only on the
+    ranking copy (the raw balance is carried on unchanged); 4.3: the copy is
+    bounded.  Reading: divide each head's balances by their largest value, so
+    the copy lies in [0, 1] (all zero when the head has no deficit).
+    """
+    m = _f64(memory)
+    out = np.zeros_like(m)
+    for h in range(m.shape[0]):
+        top = m[h].max() if m.shape[1] else 0.0
+        if top > 0.0:
+            out[h] = m[h] / top
+    return out
+
+
+def pair_means(x) -> np.ndarray:
+    """mean over query blocks i and the children j of pair p of x[h, i, j].
+
+    VASC 4.3: demand and service are averaged over query blocks and paired
+    children; A.3: a singleton is averaged over its one child.
+    """
+    x = _f64(x)
+    h_count, nbq, nb = x.shape
+    pair_of, size = block_pairs(nb)
+    out = np.zeros((h_count, size.shape[0]), dtype=np.float64)
+    for j in range(nb):
+        out[:, pair_of[j]] += x[:, :, j].sum(axis=1)
+    return out / (nbq * size)[None, :]
+
+
+def select_blocks_vasc(q, k, v, block: int, budgets, capacity: int, memory=None,
+                       value_aware: bool = True):
+    """One global layer of VASC's selection and its memory settlement.
+
+    1. pooled probabilities p (as ``selection_scores`` with lam = 0) and the
+       pair contrast rho of the pooled values;
+    2. the current demand a (``vasc_demand``);
+    3. the ranking score a_ij + M[h, pair(j)], M the ranking copy of the
+       memory carried in (VASC 4.2: memory augments the current demand;
+       reading: it is added);
+    4. a binary mask of exactly c_h blocks per row (VASC 4.2 and A.2), the
+       largest scores, ties to the lower index;
+    5. the settlement (VASC 4.3 and A.5): with D and S the pair means of the
+       demand and of the executed mask,
+           memory_out = max(0, memory_in + D - S)
+       (the accumulated deficit is clipped at zero; no memory, i.e. the
+       first layer of an inference, is all zero).
+
+    ``budgets`` holds c_h per head, 1 <= c_h <= capacity.  Returns (idx
+    [H, nb, capacity] int32: the c_h kept blocks ascending, then the last of
+    them repeated; memory_out [H, n_pairs]; a dict with probs, rho, demand,
+    mhat, score, mask, D and S).
+    """
+    sc = selection_scores(q, k, None, block, 0.0)
+    probs = sc["probs"]
+    h_count, nbq, nb = probs.shape
+    _, size = block_pairs(nb)
+    rho = pair_contrast(pool_blocks(v, block))
+    mem_in = np.zeros((h_count, size.shape[0])) if memory is None else _f64(memory)
+    demand = vasc_demand(probs, rho, budgets, value_aware)
+    mhat = memory_ranking_copy(mem_in)
+    pair_of, _ = block_pairs(nb)
+    score = demand + mhat[:, None, pair_of]
+    idx = np.zeros((h_count, nbq, capacity), dtype=np.int32)
+    mask = np.zeros_like(score)
+    for h in range(h_count):
+        c = int(budgets[h])
+        kept = topk_lowest_index(score[h], c)            # [nbq, c] ascending
+        idx[h, :, :c] = kept
+        idx[h, :, c:] = kept[:, -1:]
+        for i in range(nbq):
+            mask[h, i, kept[i]] = 1.0
+    dmean = pair_means(demand)
+    smean = pair_means(mask)
+    mem_out = np.maximum(0.0, mem_in + dmean - smean)
+    info = {"probs": probs, "rho": rho, "demand": demand, "mhat": mhat, "score": score,
+            "mask": mask, "D": dmean, "S": smean}
+    return idx, mem_out, info

@@ -73,6 +73,29 @@ MUTATIONS = {
     "a causal mask over the kept tokens":
         ("s = (q_blk @ keys.T) / math.sqrt(d)\n    m = s.max",
          "s = (q_blk @ keys.T) / math.sqrt(d)\n    s = s + np.triu(np.full(s.shape, -np.inf), 1)\n    m = s.max"),
+    "VASC contrast as the L2 norm instead of the RMS":
+        ("rho[:, p] = np.sqrt((diff * diff).sum(axis=-1) / d)",
+         "rho[:, p] = np.sqrt((diff * diff).sum(axis=-1))"),
+    "VASC sliding pairs instead of fixed ones":
+        ("diff = vbar[:, 2 * p, :] - vbar[:, 2 * p + 1, :]",
+         "diff = vbar[:, p, :] - vbar[:, p + 1, :]"),
+    "VASC singleton averaged over two children":
+        ("        size[-1] = 1", "        size[-1] = 2"),
+    "VASC demand not clipped at one":
+        ("a[h, i] = np.minimum(1.0, c * d / total)", "a[h, i] = c * d / total"),
+    "VASC demand rescaled to one instead of the capacity":
+        ("a[h, i] = np.minimum(1.0, c * d / total)", "a[h, i] = np.minimum(1.0, d / total)"),
+    "VASC contrast added to the relevance":
+        ("d = p[h, i] * factor[h]", "d = p[h, i] + factor[h]"),
+    "VASC memory normalised over all heads":
+        ("top = m[h].max() if m.shape[1] else 0.0", "top = m.max() if m.shape[1] else 0.0"),
+    "VASC memory ignored by the ranking":
+        ("score = demand + mhat[:, None, pair_of]", "score = demand + 0.0 * mhat[:, None, pair_of]"),
+    "VASC deficit not clipped at zero":
+        ("mem_out = np.maximum(0.0, mem_in + dmean - smean)", "mem_out = mem_in + dmean - smean"),
+    "VASC memory adds service and subtracts demand":
+        ("mem_out = np.maximum(0.0, mem_in + dmean - smean)",
+         "mem_out = np.maximum(0.0, mem_in - dmean + smean)"),
 }
 
 

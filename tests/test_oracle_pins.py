@@ -724,3 +724,164 @@ def test_restoration_candidates_are_the_largest_gains_and_smallest_costs():
     c = np.array([[-5.0], [-5.0], [4.0], [3.0], [4.0], [0.0]])
     kept, j0, j = oracle.restore_row(c, 2, rounds=1, cand=1)
     assert kept.tolist() == [1, 2] and j0 == 11.0 and j == 2.0
+
+
+# --------------------------------------------------------------------------
+# VASC: pair contrast, demand, memory
+# --------------------------------------------------------------------------
+
+def test_block_pairs_and_pair_contrast_closed_form():
+    # nb = 5, d = 4: pairs (0, 1), (2, 3) and the singleton 4.  Pooled values
+    # 0 and 2 (every dimension) differ by 2 in each of the 4 dimensions: RMS 2
+    # (the L2 norm would be 4).  Blocks 2 and 3 differ by 2 in one dimension:
+    # RMS sqrt(4 / 4) = 1.  The singleton has contrast 0.
+    pair_of, size = oracle.block_pairs(5)
+    assert pair_of.tolist() == [0, 0, 1, 1, 2] and size.tolist() == [2, 2, 1]
+    vbar = np.array([[[0.0, 0, 0, 0], [2, 2, 2, 2], [1, 0, 0, 0], [1, 0, 0, 2], [9, 9, 9, 9]]])
+    assert np.array_equal(oracle.pair_contrast(vbar), np.array([[2.0, 1.0, 0.0]]))
+    pair_of, size = oracle.block_pairs(4)
+    assert pair_of.tolist() == [0, 0, 1, 1] and size.tolist() == [2, 2]
+
+
+def test_pair_contrast_matches_torch_on_pooled_tokens():
+    rng = np.random.default_rng(31)
+    B, nb, H, d = 8, 7, 3, 16
+    v = rng.normal(size=(nb * B, H, d))
+    vb = torch.from_numpy(v).view(nb, B, H, d).mean(dim=1)          # [nb, H, d]
+    ref = (vb[0:nb - 1:2] - vb[1:nb:2]).pow(2).mean(dim=-1).sqrt()  # [3, H]
+    got = oracle.pair_contrast(oracle.pool_blocks(v, B))
+    np.testing.assert_allclose(got[:, :3], ref.T.numpy(), rtol=1e-13, atol=1e-15)
+    assert (got[:, 3] == 0.0).all()
+
+
+def test_demand_closed_forms():
+    # One row, nb = 4, p = (1/2, 1/4, 1/8, 1/8).
+    p = np.array([[[0.5, 0.25, 0.125, 0.125]]])
+    ones = np.ones((1, 2))
+    # Contrast one: capacity 2 gives 2 p = (1, 1/2, 1/4, 1/4), nothing clipped.
+    np.testing.assert_allclose(oracle.vasc_demand(p, ones, [2]), [[[1.0, 0.5, 0.25, 0.25]]],
+                               rtol=0, atol=1e-15)
+    np.testing.assert_allclose(oracle.vasc_demand(p, 5 * ones, [2], value_aware=False),
+                               [[[1.0, 0.5, 0.25, 0.25]]], rtol=0, atol=1e-15)
+    # Capacity 3: 3 p = (3/2, 3/4, 3/8, 3/8); the first entry clips to one.
+    np.testing.assert_allclose(oracle.vasc_demand(p, ones, [3]), [[[1.0, 0.75, 0.375, 0.375]]],
+                               rtol=0, atol=1e-15)
+    # Contrast (1, 2) multiplies: d = (1/2, 1/4, 1/4, 1/4), total 5/4, so
+    # capacity 2 gives (4/5, 2/5, 2/5, 2/5).
+    rho = np.array([[1.0, 2.0]])
+    np.testing.assert_allclose(oracle.vasc_demand(p, rho, [2]), [[[0.8, 0.4, 0.4, 0.4]]],
+                               rtol=0, atol=1e-15)
+    # A pair without contrast has no demand.
+    np.testing.assert_allclose(oracle.vasc_demand(p, np.array([[0.0, 1.0]]), [1]),
+                               [[[0.0, 0.0, 0.5, 0.5]]], rtol=0, atol=1e-15)
+
+
+def test_demand_invariants_on_tiny():
+    w, q, k, v = _tiny_inputs()
+    probs = oracle.selection_scores(q, k, None, w.block, 0.0)["probs"]
+    rho = oracle.pair_contrast(oracle.pool_blocks(v, w.block))
+    budgets = [3, 5][:probs.shape[0]]
+    a = oracle.vasc_demand(probs, rho, budgets)
+    assert (a >= 0).all() and (a <= 1.0).all()
+    for h, c in enumerate(budgets):
+        tot = a[h].sum(axis=-1)
+        assert (tot <= c + 1e-12).all()
+        d = probs[h] * rho[h][np.arange(probs.shape[-1]) // 2][None, :]
+        unclipped = (c * d / d.sum(-1, keepdims=True)).max(-1) <= 1.0
+        np.testing.assert_allclose(tot[unclipped], c, rtol=1e-13)
+
+
+def test_memory_ranking_copy_normalises_each_head_by_its_largest_balance():
+    mem = np.array([[0.0, 2.0, 1.0], [0.0, 0.0, 0.0], [3.0, 0.0, 6.0]])
+    np.testing.assert_array_equal(oracle.memory_ranking_copy(mem),
+                                  [[0.0, 1.0, 0.5], [0.0, 0.0, 0.0], [0.5, 0.0, 1.0]])
+
+
+def test_pair_means_average_over_query_blocks_and_children():
+    # H = 1, two query blocks, nb = 3: pair 0 = blocks 0 and 1, block 2 alone.
+    x = np.array([[[1.0, 2.0, 3.0], [3.0, 4.0, 5.0]]])
+    np.testing.assert_array_equal(oracle.pair_means(x), [[2.5, 4.0]])
+
+
+def _vasc_hand_inputs():
+    # B = 4, nb = 4, H = 1, d = 4.  Q = 0: every pooled logit is 0 and every
+    # probability 1/4.  Pooled values 0, 2, 0, 1: pair contrasts 2 and 1.
+    B, nb, d = 4, 4, 4
+    q = np.zeros((B * nb, 1, d))
+    k = np.random.default_rng(5).normal(size=(B * nb, 1, d))
+    v = np.zeros((B * nb, 1, d))
+    v[B:2 * B] = 2.0
+    v[3 * B:] = 1.0
+    return q, k, v, B
+
+
+def test_vasc_hand_worked_layers():
+    # Capacity 1.  Demand d = (1/4)(2, 2, 1, 1), total 3/2: a = (1/3, 1/3, 1/6,
+    # 1/6) in every row.  Pair means: D = (1/3, 1/6).
+    #  layer 1, no memory: block 0 (tie with 1, lower index); S = (1/2, 0);
+    #           memory max(0, (1/3 - 1/2, 1/6)) = (0, 1/6).
+    #  layer 2: ranking copy (0, 1), scores (1/3, 1/3, 7/6, 7/6): block 2;
+    #           S = (0, 1/2); memory (0 + 1/3, 1/6 + 1/6 - 1/2 -> 0) = (1/3, 0).
+    #  layer 3: copy (1, 0): block 0; memory (1/3 + 1/3 - 1/2, 0 + 1/6) = (1/6, 1/6).
+    #  layer 4: copy (1, 1): scores (4/3, 4/3, 7/6, 7/6): block 0;
+    #           memory (1/6 + 1/3 - 1/2, 1/6 + 1/6) = (0, 1/3).
+    q, k, v, B = _vasc_hand_inputs()
+    expect = [(0, [0.0, 1 / 6]), (2, [1 / 3, 0.0]), (0, [1 / 6, 1 / 6]), (0, [0.0, 1 / 3])]
+    mem = None
+    for layer, (block, mem_ref) in enumerate(expect):
+        idx, mem, info = oracle.select_blocks_vasc(q, k, v, B, [1], 2, mem)
+        np.testing.assert_allclose(info["demand"][0], np.tile([1 / 3, 1 / 3, 1 / 6, 1 / 6], (4, 1)),
+                                   rtol=0, atol=1e-15)
+        np.testing.assert_allclose(info["D"], [[1 / 3, 1 / 6]], rtol=0, atol=1e-15)
+        assert (idx[0] == block).all(), (layer, idx[0])       # kept block, repeated to capacity
+        np.testing.assert_allclose(mem, [mem_ref], rtol=0, atol=1e-15)
+
+
+def test_vasc_without_memory_or_contrast_is_the_pooled_topk():
+    w, q, k, v = _tiny_inputs()
+    H = q.shape[1]
+    budgets = [w.budget] * H
+    idx, _, _ = oracle.select_blocks_vasc(q, k, v, w.block, budgets, w.budget, None,
+                                          value_aware=False)
+    assert np.array_equal(idx, oracle.select_blocks(q, k, None, w.block, w.budget, 0.0))
+
+
+def test_vasc_without_memory_keeps_the_top_modulated_relevance():
+    # The clip changes no set: at most c_h entries of a row reach one, and they
+    # are the c_h largest p * rho.  Reference from torch, ranked by brute force.
+    w, q, k, v = _tiny_inputs()
+    B, H = w.block, q.shape[1]
+    budgets = [3, 5][:H]
+    idx, _, _ = oracle.select_blocks_vasc(q, k, v, B, budgets, max(budgets), None)
+    tq, tk, tv = (torch.tensor(x) for x in (q, k, v))
+    nb = tq.shape[0] // B
+    qb, kb, vb = (t.view(nb, B, *t.shape[1:]).mean(1) for t in (tq, tk, tv))
+    for h in range(H):
+        p = torch.softmax(qb[:, h] @ kb[:, h].T / 8.0, dim=-1)
+        rho = (vb[0::2, h] - vb[1::2, h]).pow(2).mean(-1).sqrt()
+        d = (p * rho.repeat_interleave(2)[None, :nb]).numpy()
+        for i in range(nb):
+            ref = _brute_force_topk(d[i], budgets[h])
+            assert idx[h, i, :budgets[h]].tolist() == list(ref)
+            assert (idx[h, i, budgets[h]:] == ref[-1]).all()
+
+
+def test_vasc_with_memory_equals_brute_force_and_conserves_service():
+    w, q, k, v = _tiny_inputs()
+    H, B = q.shape[1], w.block
+    nb = q.shape[0] // B
+    budgets = [2, 4][:H]
+    mem_in = np.random.default_rng(8).uniform(0.0, 0.3, size=(H, (nb + 1) // 2))
+    idx, mem, info = oracle.select_blocks_vasc(q, k, v, B, budgets, 4, mem_in)
+    for h in range(H):
+        for i in range(nb):
+            ref = _brute_force_topk(info["score"][h, i], budgets[h])
+            assert idx[h, i, :budgets[h]].tolist() == list(ref)
+    _, size = oracle.block_pairs(nb)
+    for h, c in enumerate(budgets):
+        # Every row executes exactly c_h children: sum_p size_p S_p = c_h.
+        assert abs((info["S"][h] * size).sum() - c) < 1e-12
+        assert (info["D"][h] * size).sum() <= c + 1e-12
+    assert (mem >= 0).all()
+    np.testing.assert_allclose(mem, np.maximum(0.0, mem_in + info["D"] - info["S"]), rtol=0,
+                               atol=0)
