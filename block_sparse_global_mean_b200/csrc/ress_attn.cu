@@ -455,7 +455,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(tS + 32, r[1]);
       tmem_ld32(tS + 64, r[2]);
       tmem_ld32(tS + 96, r[3]);
-      tmem_ld_wait();
+      tmem_ld_wait_regs(r[0]);
+      tmem_tie_regs(r[1]);
+      tmem_tie_regs(r[2]);
+      tmem_tie_regs(r[3]);
       if (kLayout) {
         if (vk0 < 64) mask_sub_block(r[0], r[1], vk0);
         if (vk1 < 64) mask_sub_block(r[2], r[3], vk1);
@@ -540,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
           tmem_ld32(tO + 32 * g, o);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(o);
 #pragma unroll
           for (int u = 0; u < 32; ++u) o[u] = __float_as_uint(__uint_as_float(o[u]) * alpha);
           tmem_st32(tO + 32 * g, o);
@@ -590,7 +593,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t oa[32], ob[32];
         tmem_ld32(tO + 32 * hc, oa);
         if (two) tmem_ld32(tO + 64 + 32 * hc, ob);
-        tmem_ld_wait();
+        tmem_ld_wait_regs(oa);
+        tmem_tie_regs(ob);
         float of[32];
 #pragma unroll
         for (int u = 0; u < 32; ++u) {

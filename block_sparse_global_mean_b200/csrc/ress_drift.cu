@@ -394,7 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t r[2][32];
           tmem_ld32(tS + 64 * hf, r[0]);
           tmem_ld32(tS + 64 * hf + 32, r[1]);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(r[0]);
+          tmem_tie_regs(r[1]);
 #pragma unroll
           for (int g = 0; g < 2; ++g) {
             const bool use = hf == 0 ? use0 : use1;
@@ -447,7 +448,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t cv[2][32];
           tmem_ld32(tmem + col + lane_off, cv[0]);
           tmem_ld32(tmem + col + lane_off + 32, cv[1]);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(cv[0]);
+          tmem_tie_regs(cv[1]);
           float2 acc[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) acc[q] = make_float2(0.f, 0.f);
@@ -518,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
           tmem_ld32(tmem + kColT + lane_off + 32 * g, tv);
-          tmem_ld_wait();
+          tmem_ld_wait_regs(tv);
 #pragma unroll
           for (int u = 0; u < 32; ++u) {
             const float x = __uint_as_float(tv[u]);
@@ -840,7 +842,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
         uint32_t r[2][32];
         tmem_ld32(tS + 64 * hf, r[0]);
         tmem_ld32(tS + 64 * hf + 32, r[1]);
-        tmem_ld_wait();
+        tmem_ld_wait_regs(r[0]);
+        tmem_tie_regs(r[1]);
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
           uint32_t pk[16];
@@ -883,7 +886,8 @@ __global__ void __launch_bounds__(kThreads2, 1)
         uint32_t cv[2][32];
         tmem_ld32(tC, cv[0]);
         tmem_ld32(tC + 32, cv[1]);
-        tmem_ld_wait();
+        tmem_ld_wait_regs(cv[0]);
+        tmem_tie_regs(cv[1]);
         tc_fence_before();
         mbar_arrive(bar_cf);
         float2 acc[4];
