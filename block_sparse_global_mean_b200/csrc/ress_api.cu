@@ -295,6 +295,40 @@ ress_status ress_select_blocks_restore(const ress_shape* shape, const void* q, c
                         static_cast<uint8_t*>(workspace), static_cast<cudaStream_t>(stream));
 }
 
+size_t ress_vasc_workspace_bytes(const ress_shape* shape) {
+  Geometry g;
+  if (check_shape(shape, &g) != RESS_OK) return 0;
+  return vasc_layout(g).total;
+}
+
+ress_status ress_select_blocks_vasc(const ress_shape* shape, const void* q, const void* k,
+                                    const void* v, const int32_t* budgets, int32_t capacity,
+                                    int32_t value_aware, int32_t reset, float* memory,
+                                    int32_t* idx, float* demand, float* service,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  Geometry g;
+  ress_status s = check_shape(shape, &g);
+  if (s != RESS_OK) return s;
+  if ((s = check_budget(g, capacity)) != RESS_OK) return s;
+  if ((value_aware != 0 && value_aware != 1) || (reset != 0 && reset != 1))
+    return RESS_ERR_INVALID_ARG;
+  if (g.nb == 0) return RESS_OK;
+  if (budgets == nullptr) return RESS_ERR_INVALID_ARG;
+  for (int h = 0; h < g.heads; ++h)
+    if (budgets[h] < 1 || budgets[h] > capacity) return RESS_ERR_INVALID_ARG;
+  if (g.nb > kMaxBlocksSelect) return RESS_ERR_UNSUPPORTED;
+  if (!q || !k || (value_aware && !v) || !memory || !idx || !workspace) return RESS_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || (v && !aligned16(v)) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u) || (reinterpret_cast<uintptr_t>(idx) & 3u) ||
+      (reinterpret_cast<uintptr_t>(memory) & 3u) || (reinterpret_cast<uintptr_t>(demand) & 3u) ||
+      (reinterpret_cast<uintptr_t>(service) & 3u))
+    return RESS_ERR_INVALID_ARG;
+  if (workspace_bytes < vasc_layout(g).total) return RESS_ERR_WORKSPACE;
+  return launch_vasc(g, q, k, v, budgets, capacity, value_aware != 0, reset != 0, memory, idx,
+                     demand, service, static_cast<uint8_t*>(workspace),
+                     static_cast<cudaStream_t>(stream));
+}
+
 size_t ress_attn_workspace_bytes(const ress_shape* shape) {
   Geometry g;
   if (check_shape(shape, &g) != RESS_OK) return 0;

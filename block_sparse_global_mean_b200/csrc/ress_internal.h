@@ -102,7 +102,8 @@ ress_status launch_attn_rows(const Geometry& g, const void* q, int64_t nq, bool 
 ress_status launch_drift(const Geometry& g, const void* q, const void* k, const void* v,
                          int budget, const int32_t* idx, const float* lse, float* drift,
                          float* set_drift, cudaStream_t st);
-// Pooling pass alone: Qbar [H][nb][64], Kbar^T and Vbar^T [H][64][nb_pad].
+// Pooling pass alone: Qbar [H][nb][64], Kbar^T and Vbar^T [H][64][nb_pad]
+// (Vbar^T only when v is not null).
 ress_status launch_pool(const Geometry& g, const void* q, const void* k, const void* v,
                         float* qbar, float* kbar_t, float* vbar_t, cudaStream_t st);
 
@@ -114,6 +115,35 @@ RestoreLayout restore_layout(const Geometry& g);
 ress_status launch_restore(const Geometry& g, const void* q, const void* k, const void* v,
                            int budget, int rounds, int cand, int32_t* idx, float* j_init,
                            float* j_final, uint8_t* ws, cudaStream_t st);
+
+// VASC selection (value-aware demand with cross-layer memory).
+// Pairs of adjacent key blocks: (nb + 1) / 2 per head, the last a singleton
+// when nb is odd.
+inline int vasc_pairs(int nb) { return (nb + 1) / 2; }
+// Inputs of the score kernel's VASC mode: c_h per head (host array of H),
+// the pair contrast and the memory's ranking copy [H][pairs], and the demand
+// (units of 2^-32) and service sums [H][pairs] it adds to (zeroed before).
+struct VascSelect {
+  const int32_t* budgets;
+  const float* rho;
+  const float* mhat;
+  unsigned long long* dsum;
+  uint32_t* ssum;
+};
+ress_status launch_score_vasc(const Geometry& g, const float* qbar, const float* kbar_t,
+                              int capacity, int32_t* idx, const VascSelect& vs,
+                              cudaStream_t st);
+// Workspace of ress_select_blocks_vasc (byte offsets): the pooled Q, K^T, V^T
+// as for the restoration, then rho, mhat [H][pairs] float32, the demand sums
+// [H][pairs] uint64 and the service counts [H][pairs] uint32.
+struct VascLayout {
+  size_t qbar, kbar_t, vbar_t, rho, mhat, dsum, ssum, total;
+};
+VascLayout vasc_layout(const Geometry& g);
+ress_status launch_vasc(const Geometry& g, const void* q, const void* k, const void* v,
+                        const int32_t* budgets, int capacity, bool value_aware, bool reset,
+                        float* memory, int32_t* idx, float* demand, float* service, uint8_t* ws,
+                        cudaStream_t st);
 
 // Workspace of the special (camera, register) rows of the layout-aware
 // attention: the gathered queries [rows_pad][H][64] bf16, their outputs and

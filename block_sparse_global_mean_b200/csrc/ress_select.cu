@@ -198,7 +198,20 @@ struct ScoreArgs {
   float tau;              // CDF threshold (cdf_counts != null)
   int32_t* cdf_counts;    // [H][nb] CDF counts, or null for the fixed budget
   int block, lay_t, lay_r, lay_s;   // per-view layout (lay_t == 0: none)
+  // VASC mode: the pair contrast and the memory's ranking copy [H][n_pairs],
+  // the demand (units of 2^-32) and service sums they add to, and c_h.
+  const float* vasc_rho;
+  const float* vasc_mhat;
+  unsigned long long* vasc_dsum;
+  uint32_t* vasc_ssum;
+  int n_pairs;
+  int vasc_budget[kMaxHeads];
 };
+
+// Modes of score_topk_kernel.
+constexpr int kModeBudget = 0;   // fixed budget: logits, or p + lambda c, or the layout ranks
+constexpr int kModeCdf = 1;      // CDF threshold
+constexpr int kModeVasc = 2;     // VASC demand plus memory, per-head budgets
 
 // Probability of logit s in units of 2^-40: p = exp(s - hi) / z in float32,
 // rounded to the nearest unit.  Sums of up to 4,096 of them are exact in 64
@@ -429,6 +442,45 @@ __device__ __noinline__ int warp_cdf_count(const float* row, int nb, unsigned lo
   return cnt_above + max(taken, 1);
 }
 
+// VASC row (one warp; row holds the pooled logits s_j of query block i).
+// With e_j = exp(s_j - max s) and rho the contrast of j's pair, the demand is
+//   a_j = min(1, e_j rho_j * c_h / sum_j e_j rho_j)
+// (the relevance p_j = e_j / sum e, times the contrast, rescaled so the row
+// totals c_h, clipped at one: VASC 4.1 and A.2); the ranking score is
+// a_j + mhat[pair(j)] (VASC 4.2), of which the c_h largest are kept (ties to
+// the lower index), listed ascending and padded with the last kept block to
+// the row length.  The demand (units of 2^-32, exact in 64 bits) and the
+// executed children are summed per pair into the CTA's counters.
+__device__ __forceinline__ void vasc_row(const ScoreArgs& a, float* row, uint32_t* whist, int h,
+                                      int i, unsigned long long* dacc, uint32_t* sacc,
+                                      int lane) {
+  const int nb = a.nb;
+  const int c = a.vasc_budget[h];
+  const float* rho = a.vasc_rho + (size_t)h * a.n_pairs;
+  const float* mhat = a.vasc_mhat + (size_t)h * a.n_pairs;
+  float m = -INFINITY;
+  for (int j = lane; j < nb; j += 32) m = fmaxf(m, row[j]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  float z = 0.f;
+  for (int j = lane; j < nb; j += 32) z += expf(row[j] - m) * rho[j >> 1];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+  const float scale = z > 0.f ? (float)c / z : 0.f;
+  for (int j = lane; j < nb; j += 32) {
+    const float dem = fminf(1.f, expf(row[j] - m) * rho[j >> 1] * scale);
+    atomicAdd(&dacc[j >> 1], __float2ull_rn(dem * 4294967296.0f));
+    row[j] = dem + mhat[j >> 1];
+  }
+  __syncwarp();
+  int32_t* out = a.idx + ((size_t)h * nb + i) * a.budget;
+  warp_topk_row_binned(row, nb, c, whist, out, lane);
+  __syncwarp();
+  const int32_t last = out[c - 1];
+  for (int r = c + lane; r < a.budget; r += 32) out[r] = last;
+  for (int r = lane; r < c; r += 32) atomicAdd(&sacc[out[r] >> 1], 1u);
+}
+
 // CTA = one head and R consecutive query blocks.  The pooled keys stream
 // through a ring of 16 KB shared-memory stages, each [4 d][1024 keys] fp32,
 // filled by bulk copies that the producer (the last warp) issues as soon as
@@ -457,7 +509,7 @@ struct ScoreCfg {
 
 // Registers are capped at 128 so that four warps of one SM sub-partition fit
 // its register file (4 x 32 x 128 = 16,384).
-template <int R, bool kCdf>
+template <int R, int kMode>
 __global__ void __maxnreg__(128) score_topk_kernel(const ScoreArgs a) {
   using C = ScoreCfg<R>;
   constexpr int TK = kScoreTK, TD = kScoreTD;
@@ -469,6 +521,9 @@ __global__ void __maxnreg__(128) score_topk_kernel(const ScoreArgs a) {
   const int nb = a.nb, nb_pad = a.nb_pad, rs = a.row_stride;
   uint64_t* bars = reinterpret_cast<uint64_t*>(scores + (size_t)R * rs);   // full[S], empty[S]
   int* abortf = reinterpret_cast<int*>(bars + 2 * S);
+  // VASC mode: this CTA's demand sums [n_pairs] and service counts [n_pairs].
+  unsigned long long* dacc = reinterpret_cast<unsigned long long*>(bars + 2 * S + 2);
+  uint32_t* sacc = reinterpret_cast<uint32_t*>(dacc + a.n_pairs);
 
   const int h = blockIdx.x / a.tiles_per_head;
   const int i0 = (blockIdx.x % a.tiles_per_head) * R;
@@ -491,6 +546,12 @@ __global__ void __maxnreg__(128) score_topk_kernel(const ScoreArgs a) {
   for (int e = tid; e < R * kHeadDim; e += C::kThreads) {
     const int r = e / kHeadDim, d = e % kHeadDim;
     qs[d * R + r] = (i0 + r < nb) ? a.qbar[((size_t)h * nb + i0 + r) * kHeadDim + d] : 0.f;
+  }
+  if constexpr (kMode == kModeVasc) {
+    for (int p = tid; p < a.n_pairs; p += C::kThreads) {
+      dacc[p] = 0ull;
+      sacc[p] = 0u;
+    }
   }
   __syncthreads();
 
@@ -589,6 +650,22 @@ __global__ void __maxnreg__(128) score_topk_kernel(const ScoreArgs a) {
     }
   }
   __syncthreads();
+  if constexpr (kMode == kModeVasc) {
+    if (*abortf != 0) return;   // read after the barrier: the same for every thread
+    if (warp < R && i0 + warp < nb)
+      vasc_row(a, scores + (size_t)warp * rs,
+               reinterpret_cast<uint32_t*>(stages) + warp * kWarpScratchStride, h, i0 + warp,
+               dacc, sacc, lane);
+    __syncthreads();
+    // This CTA's sums join the head's totals (integer adds: the totals do not
+    // depend on the order of the CTAs).
+    for (int p = tid; p < a.n_pairs; p += C::kThreads) {
+      const size_t at = (size_t)h * a.n_pairs + p;
+      if (dacc[p] != 0ull) atomicAdd(&a.vasc_dsum[at], dacc[p]);
+      if (sacc[p] != 0u) atomicAdd(&a.vasc_ssum[at], sacc[p]);
+    }
+    return;
+  }
   if (*abortf != 0 || warp >= R) return;
   // One warp per row; the stage buffers now hold each row warp's scratch.
   const int i = i0 + warp;
@@ -596,7 +673,7 @@ __global__ void __maxnreg__(128) score_topk_kernel(const ScoreArgs a) {
   uint32_t* whist = reinterpret_cast<uint32_t*>(stages) + warp * kWarpScratchStride;
   float* row = scores + (size_t)warp * rs;
   int32_t* out = a.idx + ((size_t)h * nb + i) * a.budget;
-  if constexpr (kCdf) {
+  if constexpr (kMode == kModeCdf) {
     // CDF threshold: the count, then the exact top min(count, capacity) of the
     // logits (the probabilities' order), padded with the last kept block.
     // At least one unit: every row keeps at least its top block.
@@ -643,10 +720,11 @@ __global__ void __maxnreg__(128) score_topk_kernel(const ScoreArgs a) {
 // Shared memory of score_topk_kernel<R> with `stages` ring stages and score
 // rows of `row_stride` floats.
 template <int R>
-size_t score_smem_bytes(int stages, int row_stride) {
+size_t score_smem_bytes(int stages, int row_stride, int n_pairs = 0) {
   return (size_t)stages * kStageBytes +
          sizeof(float) * ((size_t)kHeadDim * R + (size_t)R * row_stride) +
-         2 * sizeof(uint64_t) * (size_t)stages + 16;
+         2 * sizeof(uint64_t) * (size_t)stages + 16 +
+         (sizeof(unsigned long long) + sizeof(uint32_t)) * (size_t)n_pairs;
 }
 
 constexpr size_t kMaxSmem = 227 * 1024;
@@ -654,31 +732,34 @@ constexpr int kMaxStages = 6;
 
 // Deepest ring (up to kMaxStages) that fits; 0 if fewer than `min_stages` fit.
 template <int R>
-int score_stages(int row_stride, int min_stages) {
+int score_stages(int row_stride, int min_stages, int n_pairs = 0) {
   for (int s = kMaxStages; s >= min_stages; --s)
-    if (score_smem_bytes<R>(s, row_stride) <= kMaxSmem) return s;
+    if (score_smem_bytes<R>(s, row_stride, n_pairs) <= kMaxSmem) return s;
   return 0;
 }
 
-template <int R, bool kCdf>
+template <int R, int kMode>
 ress_status launch_score_mode(const ScoreArgs& a0, int stages, cudaStream_t st) {
   ScoreArgs a = a0;
   a.tiles_per_head = (a.nb + R - 1) / R;
   a.stages = stages;
-  const size_t smem = score_smem_bytes<R>(stages, a.row_stride);
+  const size_t smem =
+      score_smem_bytes<R>(stages, a.row_stride, kMode == kModeVasc ? a.n_pairs : 0);
   if (ress_status st_ = record_cuda(cudaFuncSetAttribute(
-          score_topk_kernel<R, kCdf>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
+          score_topk_kernel<R, kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
     return st_;
-  score_topk_kernel<R, kCdf><<<a.heads * a.tiles_per_head, ScoreCfg<R>::kThreads, smem, st>>>(a);
+  score_topk_kernel<R, kMode><<<a.heads * a.tiles_per_head, ScoreCfg<R>::kThreads, smem, st>>>(a);
   return record_cuda(cudaGetLastError());
 }
 
-// The CDF mode is a separate instantiation, so that its code does not weigh on
-// the register allocation and code layout of the fixed-budget kernel.
+// The CDF and VASC modes are separate instantiations, so that their code does
+// not weigh on the register allocation and code layout of the fixed-budget
+// kernel.
 template <int R>
 ress_status launch_score(const ScoreArgs& a, int stages, cudaStream_t st) {
-  return a.cdf_counts != nullptr ? launch_score_mode<R, true>(a, stages, st)
-                                 : launch_score_mode<R, false>(a, stages, st);
+  if (a.vasc_rho != nullptr) return launch_score_mode<R, kModeVasc>(a, stages, st);
+  return a.cdf_counts != nullptr ? launch_score_mode<R, kModeCdf>(a, stages, st)
+                                 : launch_score_mode<R, kModeBudget>(a, stages, st);
 }
 
 // Exact top-k of the rows that the tensor-core kernel handed over (its check
@@ -739,7 +820,7 @@ ress_status launch_pool(const Geometry& g, const void* q, const void* k, const v
   const int epv = g.f32 ? 4 : 8;
   pa.vpr = g.heads * kHeadDim / epv;
   const int phases = pa.vpr >= 256 ? 1 : 256 / pa.vpr;
-  const dim3 grid(g.nb, 3);
+  const dim3 grid(g.nb, v != nullptr ? 3 : 2);
   const int threads = pa.vpr * phases;
   const size_t red = phases > 1 ? sizeof(float) * (size_t)phases * pa.vpr * epv : 0;
   if (g.f32)
@@ -747,6 +828,35 @@ ress_status launch_pool(const Geometry& g, const void* q, const void* k, const v
   else
     pool_kernel<__nv_bfloat16><<<grid, threads, red, st>>>(pa);
   return record_cuda(cudaGetLastError());
+}
+
+ress_status launch_score_vasc(const Geometry& g, const float* qbar, const float* kbar_t,
+                              int capacity, int32_t* idx, const VascSelect& vs,
+                              cudaStream_t st) {
+  ScoreArgs sa{};
+  sa.err = device_error_ptr();
+  if (sa.err == nullptr) return RESS_ERR_CUDA;
+  sa.qbar = qbar;
+  sa.kbar_t = kbar_t;
+  sa.idx = idx;
+  sa.heads = g.heads;
+  sa.nb = g.nb;
+  sa.nb_pad = g.nb_pad;
+  sa.budget = capacity;
+  sa.block = g.block;
+  sa.row_stride = (g.nb + 3) & ~3;
+  sa.vasc_rho = vs.rho;
+  sa.vasc_mhat = vs.mhat;
+  sa.vasc_dsum = vs.dsum;
+  sa.vasc_ssum = vs.ssum;
+  sa.n_pairs = vasc_pairs(g.nb);
+  for (int h = 0; h < g.heads; ++h) sa.vasc_budget[h] = vs.budgets[h];
+  // As for the fixed budget, with the CTA's pair counters next to the rows.
+  const int s16 = score_stages<16>(sa.row_stride, 4, sa.n_pairs);
+  if (s16 != 0) return launch_score<16>(sa, s16, st);
+  const int s8 = score_stages<8>(sa.row_stride, 2, sa.n_pairs);
+  if (s8 == 0) return RESS_ERR_UNSUPPORTED;
+  return launch_score<8>(sa, s8, st);
 }
 
 ress_status launch_topk_fallback(const Geometry& g, int budget, int32_t* idx, uint8_t* ws,

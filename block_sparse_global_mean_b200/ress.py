@@ -92,6 +92,11 @@ lib.ress_restore_workspace_bytes.argtypes = [_SHAPE]
 lib.ress_select_blocks_restore.restype = ctypes.c_int
 lib.ress_select_blocks_restore.argtypes = [_SHAPE, _P, _P, _P, ctypes.c_int32, ctypes.c_int32,
                                            ctypes.c_int32, _P, _P, _P, _P, ctypes.c_size_t, _P]
+lib.ress_vasc_workspace_bytes.restype = ctypes.c_size_t
+lib.ress_vasc_workspace_bytes.argtypes = [_SHAPE]
+lib.ress_select_blocks_vasc.restype = ctypes.c_int
+lib.ress_select_blocks_vasc.argtypes = [_SHAPE, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_int32,
+                                        ctypes.c_int32, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]
 lib.ress_validate_idx.restype = ctypes.c_int
 lib.ress_validate_idx.argtypes = [_SHAPE, ctypes.c_int32, _P, _P]
 lib.ress_check_device_errors.restype = ctypes.c_int
@@ -478,6 +483,66 @@ def ress_select_blocks_restore(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor
                  _stream_ptr(stream, q.device))
     _check(status, "ress_select_blocks_restore")
     return idx, drift_init, drift_final
+
+
+def vasc_pairs(nb: int) -> int:
+    """Memory entries per head of the VASC selection: one per fixed pair of
+    neighbouring key blocks, the last a singleton when nb is odd."""
+    return (nb + 1) // 2
+
+
+def ress_select_blocks_vasc(q: torch.Tensor, k: torch.Tensor, v: Optional[torch.Tensor],
+                            budgets, block: int, capacity: Optional[int] = None,
+                            memory: Optional[torch.Tensor] = None, value_aware: bool = True,
+                            reset: Optional[bool] = None, idx: Optional[torch.Tensor] = None,
+                            demand: Optional[torch.Tensor] = None,
+                            service: Optional[torch.Tensor] = None,
+                            workspace: Optional[torch.Tensor] = None,
+                            stream: Optional[torch.cuda.Stream] = None
+                            ) -> Tuple[torch.Tensor, torch.Tensor, Optional[torch.Tensor],
+                                       Optional[torch.Tensor]]:
+    """VASC selection of one global layer: returns (idx [H, nb, capacity]
+    int32, memory [H, pairs] float32 settled in place, demand, service).
+
+    ``budgets`` holds c_h for every head (an int applies to all); capacity
+    defaults to the largest.  Without ``memory`` a zeroed one is made and
+    ``reset`` defaults to True (the first global layer); with one, ``reset``
+    defaults to False.  ``demand`` / ``service`` ([H, pairs] float32) are
+    filled when given.
+    """
+    _check_inputs(q, k, v)
+    if value_aware and v is None:
+        raise ValueError("the value contrast needs v (or value_aware=False)")
+    sh = _shape_of(q, block)
+    n, h = q.shape[0], q.shape[1]
+    nb = n // block
+    pairs = vasc_pairs(nb)
+    per_head = [int(budgets)] * h if isinstance(budgets, int) else [int(b) for b in budgets]
+    if len(per_head) != h:
+        raise ValueError(f"budgets needs {h} entries, got {len(per_head)}")
+    cap = max(per_head) if capacity is None else int(capacity)
+    if memory is None:
+        memory = torch.zeros((h, pairs), dtype=torch.float32, device=q.device)
+        reset = True if reset is None else reset
+    reset = False if reset is None else reset
+    if idx is None:
+        idx = torch.empty((h, nb, max(cap, 1)), dtype=torch.int32, device=q.device)
+    _check_buffer(memory, (h, pairs), torch.float32, q.device, "memory")
+    _check_buffer(idx, (h, nb, max(cap, 1)), torch.int32, q.device, "idx")
+    for name, t in (("demand", demand), ("service", service)):
+        if t is not None:
+            _check_buffer(t, (h, pairs), torch.float32, q.device, name)
+    _check_workspace(workspace, q.device)
+    need = int(lib.ress_vasc_workspace_bytes(ctypes.byref(sh)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    host_budgets = (ctypes.c_int32 * h)(*per_head)
+    status = _on(q.device, lib.ress_select_blocks_vasc, ctypes.byref(sh), _ptr(q), _ptr(k),
+                 _ptr(v), ctypes.cast(host_budgets, _P), cap, int(bool(value_aware)),
+                 int(bool(reset)), _ptr(memory), _ptr(idx), _ptr(demand), _ptr(service),
+                 _ptr(workspace), workspace.numel(), _stream_ptr(stream, q.device))
+    _check(status, "ress_select_blocks_vasc")
+    return idx, memory, demand, service
 
 
 def ress_validate_idx(idx: torch.Tensor, n: int, block: int,

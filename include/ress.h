@@ -252,6 +252,64 @@ ress_status ress_select_blocks_restore(const ress_shape* shape, const void* q, c
                                        size_t workspace_bytes, void* stream);
 
 /*
+ * Workspace bytes of ress_select_blocks_vasc (0 if the shape is invalid):
+ * Qbar [H][nb][64], Kbar^T and Vbar^T [H][64][nb_pad] float32, then per pair
+ * the contrast and the memory's ranking copy (float32), the demand sum
+ * (uint64) and the service count (uint32), [H][(nb + 1) / 2] each; every
+ * array 256-byte aligned.
+ */
+size_t ress_vasc_workspace_bytes(const ress_shape* shape);
+
+/*
+ * Stage 1 as VASC selects it, one global layer per call: value-aware demand,
+ * a binary mask of exactly c_h blocks per row, and the cross-layer memory
+ * settled by what was executed (VASC 4.1, 4.2, 4.3, A.1 - A.5; per-head
+ * budgets c_h as in ReSS Fig. 3 and Table 2).
+ *
+ * Key blocks form fixed pairs of neighbours (2p, 2p+1), p < (nb + 1) / 2; an
+ * odd final block is a singleton.  For head h and query block i, with p_ij
+ * the pooled probabilities of ress_select_blocks:
+ *   rho_p  = sqrt( (1/64) sum_d (Vbar_2p,d - Vbar_2p+1,d)^2 ), 0 for a
+ *            singleton (the RMS contrast of the pair); 1 for every pair when
+ *            value_aware == 0 (the contrast set to one);
+ *   a_ij   = min(1, c_h * p_ij rho_pair(j) / sum_j p_ij rho_pair(j))
+ *            (0 when the sum is 0): the demand, rescaled to the capacity and
+ *            clipped at one;
+ *   mhat_p = memory_p / max over the head's pairs (0 when that is 0): the
+ *            ranking copy of the memory;
+ *   kept   = the c_h largest a_ij + mhat_pair(j), ties to the lower index.
+ * Then, with D_p and S_p the means of a_ij and of the kept mask over all query
+ * blocks i and the children j of pair p,
+ *   memory_p <- max(0, memory_p + D_p - S_p).
+ * How the contrast modulates the relevance (a factor), how memory enters the
+ * ranking (added), how it is normalised (by the head's largest balance) and
+ * the rescaling (proportional, one clip) are this library's readings.
+ *
+ *   v            [N][H][64], needed when value_aware != 0 (else may be NULL).
+ *   budgets      HOST array of H int32: c_h, 1 <= c_h <= capacity.
+ *   capacity     1 <= capacity <= nb: the length of every idx row.
+ *   value_aware  1: contrast on; 0: contrast one.
+ *   reset        1: the memory is taken as zero on entry (the first global
+ *                layer of an inference, or a changed layout); 0: carried in.
+ *   memory       in/out, device [H][(nb + 1) / 2] float32 (>= 0).
+ *   idx          out, [H][nb][capacity] int32: row (h, i) holds its c_h kept
+ *                blocks ascending, then the last of them repeated, a valid
+ *                kept list for ress_block_sparse_attn with budget = capacity.
+ *   demand       out, [H][(nb + 1) / 2] float32, D; or NULL.
+ *   service      out, [H][(nb + 1) / 2] float32, S; or NULL.
+ *   workspace    ress_vasc_workspace_bytes(shape) bytes, 256-byte aligned.
+ *   Supported sizes: nb <= 4096.  The demand sums are exact in fixed point
+ *   (units of 2^-32), so memory, demand and service do not depend on the
+ *   order of the kernel's blocks; the scores are float32, so a ranking
+ *   decision between two values equal to float32 rounding may go either way.
+ */
+ress_status ress_select_blocks_vasc(const ress_shape* shape, const void* q, const void* k,
+                                    const void* v, const int32_t* budgets, int32_t capacity,
+                                    int32_t value_aware, int32_t reset, float* memory,
+                                    int32_t* idx, float* demand, float* service,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Workspace bytes that ress_block_sparse_attn and ress_block_drift need:
  * 0 for bf16 inputs; 3 * N * H * 64 * 2 for float32 inputs (bf16 copies of
  * q, k and v).

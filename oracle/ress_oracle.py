@@ -694,7 +694,11 @@ def select_blocks_vasc(q, k, v, block: int, budgets, capacity: int, memory=None,
     probs = sc["probs"]
     h_count, nbq, nb = probs.shape
     _, size = block_pairs(nb)
-    rho = pair_contrast(pool_blocks(v, block))
+    if value_aware:
+        assert v is not None, "the value contrast needs V"
+        rho = pair_contrast(pool_blocks(v, block))
+    else:
+        rho = np.ones((h_count, size.shape[0]), dtype=np.float64)   # unused: contrast one
     mem_in = np.zeros((h_count, size.shape[0])) if memory is None else _f64(memory)
     demand = vasc_demand(probs, rho, budgets, value_aware)
     mhat = memory_ranking_copy(mem_in)

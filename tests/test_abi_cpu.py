@@ -291,3 +291,45 @@ def test_restore_rejects_bad_arguments_on_the_host(ress):
     assert call(ws_bytes=16) == ress.RESS_ERR_WORKSPACE
     # Qbar, Kbar^T and Vbar^T (nb_pad = 256)
     assert lib.ress_restore_workspace_bytes(ctypes.byref(sh)) == 4 * 2 * 8 * 64 + 2 * 4 * 2 * 64 * 256
+
+
+@no_gpu_only
+def test_vasc_rejects_bad_arguments_on_the_host(ress):
+    lib = ress.lib
+    sh = _shape(ress)                                              # H = 2, nb = 8
+
+    def call(budgets=(2, 3), cap=4, va=1, reset=0, q=FAKE, v=FAKE, mem=FAKE, dem=None,
+             ws_bytes=1 << 30):
+        arr = None if budgets is None else (ctypes.c_int32 * len(budgets))(*budgets)
+        return lib.ress_select_blocks_vasc(ctypes.byref(sh), q, FAKE, v,
+                                           None if arr is None else ctypes.cast(arr, ctypes.c_void_p),
+                                           cap, va, reset, mem, FAKE, dem, None, FAKE_WS, ws_bytes,
+                                           None)
+    assert call(budgets=None) == ress.RESS_ERR_INVALID_ARG
+    assert call(budgets=(0, 3)) == ress.RESS_ERR_INVALID_ARG
+    assert call(budgets=(2, 5)) == ress.RESS_ERR_INVALID_ARG      # above the capacity
+    assert call(cap=0) == ress.RESS_ERR_INVALID_ARG
+    assert call(cap=9) == ress.RESS_ERR_INVALID_ARG               # above nb
+    assert call(va=2) == ress.RESS_ERR_INVALID_ARG
+    assert call(reset=-1) == ress.RESS_ERR_INVALID_ARG
+    assert call(v=None) == ress.RESS_ERR_INVALID_ARG              # the contrast needs V
+    assert call(mem=None) == ress.RESS_ERR_INVALID_ARG
+    assert call(q=FAKE + 4) == ress.RESS_ERR_INVALID_ARG
+    assert call(mem=FAKE + 2) == ress.RESS_ERR_INVALID_ARG
+    assert call(dem=FAKE + 2) == ress.RESS_ERR_INVALID_ARG
+    assert call(ws_bytes=16) == ress.RESS_ERR_WORKSPACE
+    assert lib.ress_select_blocks_vasc(None, FAKE, FAKE, FAKE, None, 4, 1, 0, FAKE, FAKE, None,
+                                       None, FAKE_WS, 1 << 30, None) == ress.RESS_ERR_INVALID_ARG
+    # Qbar; Kbar^T and Vbar^T (nb_pad = 256); rho, mhat, demand sums and
+    # service counts for 2 x 4 pairs, each padded to 256 bytes.
+    assert lib.ress_vasc_workspace_bytes(ctypes.byref(sh)) == \
+        4 * 2 * 8 * 64 + 2 * 4 * 2 * 64 * 256 + 4 * 256
+
+
+def test_vasc_binding_checks_its_buffers_before_the_library(ress):
+    q = torch.zeros(512, 2, 64)
+    with pytest.raises(ValueError):
+        ress.ress_select_blocks_vasc(q, q, None, [2, 3], 64)      # contrast without V
+    with pytest.raises(ValueError):
+        ress.ress_select_blocks_vasc(q, q, q, [2, 3, 4], 64)      # one budget per head
+    assert ress.vasc_pairs(8) == 4 and ress.vasc_pairs(9) == 5
