@@ -567,6 +567,31 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         cdf_ms = e0.elapsed_time(e1) / 5
         del counts, cidx, ws_cdf
 
+    # One VASC layer (value-aware demand, the same budget for every head,
+    # memory carried across the five timed calls) on the same input.
+    vasc_ms = None
+    if rank == 0 and not args.no_extra:
+        pairs = ress.vasc_pairs(nb)
+        mem = torch.zeros((H, pairs), dtype=torch.float32, device=dev)
+        vidx = torch.empty((H, nb, w.budget), dtype=torch.int32, device=dev)
+        ws_v = torch.empty(max(1, ress.vasc_workspace_bytes(w.n_tokens, H, w.block, q.dtype)),
+                           dtype=torch.uint8, device=dev)
+        ress.ress_select_blocks_vasc(q, k, v, w.budget, w.block, memory=mem, reset=True, idx=vidx,
+                                     workspace=ws_v, stream=stream)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(5):
+            ress.ress_select_blocks_vasc(q, k, v, w.budget, w.block, memory=mem, idx=vidx,
+                                         workspace=ws_v, stream=stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        vasc_ms = e0.elapsed_time(e1) / 5
+        del mem, vidx, ws_v
+        status, detail = ress.ress_check_device_errors(stream, dev)
+        if status != 0:
+            raise RuntimeError(f"device error {status} (detail {detail}) in the CDF / VASC stages")
+
     extra = None
     if rank == 0 and world == 1 and not args.no_extra and w.name == "views100":
         del q, k, v
@@ -630,6 +655,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if cdf_ms is not None:
         line["stages"]["select_cdf_ms"] = cdf_ms
         line["stages"]["select_cdf"] = "CDF-threshold selection, tau 0.9, capacity = budget"
+    if vasc_ms is not None:
+        line["stages"]["select_vasc_ms"] = vasc_ms
+        line["stages"]["select_vasc"] = ("VASC layer: pair contrast, demand, memory, per-head "
+                                         "budgets = budget; pooling of Q, K, V included")
     if w.drift:
         line["stages"]["drift_ms"] = dr_ms
         line["stages"]["drift_tflops"] = w.drift_flops() * H / w.heads / (dr_ms / 1e3) / 1e12

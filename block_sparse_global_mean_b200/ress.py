@@ -202,6 +202,11 @@ def select_workspace_bytes(n: int, heads: int, block: int, dtype: torch.dtype, l
     return int(lib.ress_select_workspace_bytes(ctypes.byref(sh), ctypes.c_float(lam)))
 
 
+def vasc_workspace_bytes(n: int, heads: int, block: int, dtype: torch.dtype) -> int:
+    sh = make_shape(n, heads, block, dtype)
+    return int(lib.ress_vasc_workspace_bytes(ctypes.byref(sh)))
+
+
 def attn_workspace_bytes(n: int, heads: int, block: int, dtype: torch.dtype) -> int:
     sh = make_shape(n, heads, block, dtype)
     return int(lib.ress_attn_workspace_bytes(ctypes.byref(sh)))
