@@ -588,6 +588,40 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         torch.cuda.synchronize(dev)
         vasc_ms = e0.elapsed_time(e1) / 5
         del mem, vidx, ws_v
+
+    # The layout-aware path (VGGT views of 1,408 tokens: 1,374 real, 5 special)
+    # and the restoration-based selection (4 rounds, 8 candidates per side) on
+    # the same input, when it is the 100-view workload.
+    layout_ms = restore_ms = None
+    if rank == 0 and not args.no_extra and w.name == "views100" and args.shard == "none":
+        lay = (1408, 1374, 5)
+        lidx = ress.ress_select_blocks_layout(q, k, w.budget, w.block, lay, stream=stream)
+        lout, llse = ress.ress_block_sparse_attn_layout(q, k, v, lidx, w.block, lay, stream=stream)
+
+        def _timed(fn, reps):
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(reps):
+                fn()
+            a1.record(stream)
+            torch.cuda.synchronize(dev)
+            return a0.elapsed_time(a1) / reps
+
+        layout_ms = {
+            "select": _timed(lambda: ress.ress_select_blocks_layout(
+                q, k, w.budget, w.block, lay, idx=lidx, stream=stream), 5),
+            "attn": _timed(lambda: ress.ress_block_sparse_attn_layout(
+                q, k, v, lidx, w.block, lay, out=lout, lse=llse, stream=stream), 3),
+        }
+        ridx = torch.empty((H, nb, w.budget), dtype=torch.int32, device=dev)
+        ress.ress_select_blocks_restore(q, k, v, w.budget, w.block, 4, 8, idx=ridx, stream=stream)
+        restore_ms = _timed(lambda: ress.ress_select_blocks_restore(
+            q, k, v, w.budget, w.block, 4, 8, idx=ridx, stream=stream), 2)
+        del lidx, lout, llse, ridx
+        status, detail = ress.ress_check_device_errors(stream, dev)
+        if status != 0:
+            raise RuntimeError(f"device error {status} (detail {detail}) in the layout / restore stages")
         status, detail = ress.ress_check_device_errors(stream, dev)
         if status != 0:
             raise RuntimeError(f"device error {status} (detail {detail}) in the CDF / VASC stages")
@@ -659,6 +693,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         line["stages"]["select_vasc_ms"] = vasc_ms
         line["stages"]["select_vasc"] = ("VASC layer: pair contrast, demand, memory, per-head "
                                          "budgets = budget; pooling of Q, K, V included")
+    if layout_ms is not None:
+        line["stages"]["layout_select_ms"] = layout_ms["select"]
+        line["stages"]["layout_attn_ms"] = layout_ms["attn"]
+        line["stages"]["layout"] = ("views of 1,408 tokens, 1,374 real, 5 special: padding masked, "
+                                    "special queries dense, special rows gathered and scattered")
+    if restore_ms is not None:
+        line["stages"]["select_restore_ms"] = restore_ms
+        line["stages"]["select_restore"] = "drift score + 4 restoration rounds, 8 candidates per side"
     if w.drift:
         line["stages"]["drift_ms"] = dr_ms
         line["stages"]["drift_tflops"] = w.drift_flops() * H / w.heads / (dr_ms / 1e3) / 1e12

@@ -76,6 +76,31 @@ __device__ __forceinline__ void warp_best(float& v, int& j) {
   }
 }
 
+// out[j] = sum_d x[d] * mt[d][j] for every j < nb (d ascending, float32
+// FMA): lane l takes blocks l, l + 32, l + 64, l + 96 of each group of 128 at
+// once, four independent chains with their loads in flight together.  Loads
+// past nb stay inside the padded row (index clamped to nb_pad - 1) and are
+// not stored.
+__device__ __forceinline__ void dots4(const float* x, const float* __restrict__ mt, int nb_pad,
+                                      int nb, float* out, int lane) {
+  for (int j0 = lane; j0 < nb; j0 += 128) {
+    int jj[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) jj[u] = min(j0 + 32 * u, nb_pad - 1);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int d = 0; d < kHeadDim; ++d) {
+      const float xd = x[d];
+      const float* row = mt + (size_t)d * nb_pad;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[u] = fmaf(xd, row[jj[u]], acc[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      if (j0 + 32 * u < nb) out[j0 + 32 * u] = acc[u];
+  }
+}
+
 __global__ void __launch_bounds__(32 * kRsMaxWarps) restore_kernel(const RestoreArgs a) {
   extern __shared__ __align__(16) float rsm[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -106,12 +131,10 @@ __global__ void __launch_bounds__(32 * kRsMaxWarps) restore_kernel(const Restore
   __syncwarp();
 
   // Pooled logits (d ascending, float32 FMA, exact 1/8) and probabilities.
+  dots4(T, kt, a.nb_pad, nb, p, lane);
   float m = -INFINITY;
   for (int j = lane; j < nb; j += 32) {
-    float s = 0.f;
-#pragma unroll 8
-    for (int d = 0; d < kHeadDim; ++d) s = fmaf(T[d], kt[(size_t)d * a.nb_pad + j], s);
-    s *= 0.125f;
+    const float s = p[j] * 0.125f;
     p[j] = s;
     m = fmaxf(m, s);
   }
@@ -168,12 +191,7 @@ __global__ void __launch_bounds__(32 * kRsMaxWarps) restore_kernel(const Restore
     T[lane] = t0;
     T[lane + 32] = t1;
     __syncwarp();
-    for (int j = lane; j < nb; j += 32) {
-      float s = 0.f;
-#pragma unroll 8
-      for (int d = 0; d < kHeadDim; ++d) s = fmaf(T[d], vt[(size_t)d * a.nb_pad + j], s);
-      dot[j] = s;
-    }
+    dots4(T, vt, a.nb_pad, nb, dot, lane);
     __syncwarp();
     // Candidates: the dropped blocks of largest gain 2 <T, c_b> - |c_b|^2 and
     // the kept blocks of smallest cost 2 <T, c_a> + |c_a|^2.

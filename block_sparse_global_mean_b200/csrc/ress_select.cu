@@ -462,15 +462,28 @@ __device__ __forceinline__ void vasc_row(const ScoreArgs& a, float* row, uint32_
   for (int j = lane; j < nb; j += 32) m = fmaxf(m, row[j]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  // e_j rho_j replaces the logit (one exponential per entry).
   float z = 0.f;
-  for (int j = lane; j < nb; j += 32) z += expf(row[j] - m) * rho[j >> 1];
+  for (int j = lane; j < nb; j += 32) {
+    const float w = expf(row[j] - m) * rho[j >> 1];
+    row[j] = w;
+    z += w;
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
   const float scale = z > 0.f ? (float)c / z : 0.f;
-  for (int j = lane; j < nb; j += 32) {
-    const float dem = fminf(1.f, expf(row[j] - m) * rho[j >> 1] * scale);
-    atomicAdd(&dacc[j >> 1], __float2ull_rn(dem * 4294967296.0f));
-    row[j] = dem + mhat[j >> 1];
+  // Lanes 2l and 2l + 1 hold the two children of one pair (32 is even), so
+  // the even lane adds both demands to the pair's counter.
+  for (int j0 = 0; j0 < nb; j0 += 32) {
+    const int j = j0 + lane;
+    unsigned long long fx = 0ull;
+    if (j < nb) {
+      const float dem = fminf(1.f, row[j] * scale);
+      fx = __float2ull_rn(dem * 4294967296.0f);
+      row[j] = dem + mhat[j >> 1];
+    }
+    fx += __shfl_xor_sync(0xffffffffu, fx, 1);
+    if ((lane & 1) == 0 && j < nb) atomicAdd(&dacc[j >> 1], fx);
   }
   __syncwarp();
   int32_t* out = a.idx + ((size_t)h * nb + i) * a.budget;
