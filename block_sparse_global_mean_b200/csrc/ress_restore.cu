@@ -14,9 +14,12 @@
 // swapped if that is below |T|; otherwise restoration stops.  The result is
 // the last accepted set, which has the smallest drift of all rounds.
 //
-// One warp per row; the row's probabilities, drift scores, value norms and
-// candidate contributions live in shared memory, the pooled keys and values
-// (transposed, [64][nb_pad] per head) are read from the workspace.
+// One CTA of four warps per row: the passes over the row's key blocks (logits,
+// values, the per-round products with T) are split over all 128 threads, the
+// row's probabilities, drift scores, value norms and candidate contributions
+// live in shared memory, and the pooled keys and values (transposed,
+// [64][nb_pad] per head) are read from the workspace.  Sums across threads
+// follow a fixed order, so the result is deterministic.
 //
 // Sources: ReSS (thelatestinai.com) Abstract and Fig. 1 (drift: the shift a
 // masked block leaves in the residual stream; the drift of a drop set depends
@@ -33,7 +36,8 @@ namespace ress {
 
 namespace {
 
-constexpr int kRsMaxWarps = 4;       // rows per CTA, at most
+constexpr int kRsThreads = 128;      // one row per CTA
+constexpr int kRsWarps = kRsThreads / 32;
 constexpr int kRsMaxCand = 16;
 
 struct RestoreArgs {
@@ -45,7 +49,6 @@ struct RestoreArgs {
   float* j_final;        // [H][nb] or null
   int heads, nb, nb_pad, budget, rounds, cand;
   int row_stride;        // floats of one shared-memory row (nb rounded up to 4)
-  int warp_floats;       // floats of one warp's shared memory
 };
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -59,34 +62,72 @@ __device__ __forceinline__ float warp_add(float v) {
   return v;
 }
 
-// Warp-wide best (value, index): the largest (kLargest) or smallest value,
-// ties to the lower index; entries with index INT_MAX do not count.
+// (value, index) v beats (ov, oj): the larger (kLargest) or smaller value,
+// ties to the lower index; index INT_MAX is no entry.
+template <bool kLargest>
+__device__ __forceinline__ bool beats(float v, int j, float ov, int oj) {
+  if (j == INT_MAX) return false;
+  if (oj == INT_MAX) return true;
+  return (kLargest ? v > ov : v < ov) || (v == ov && j < oj);
+}
+
 template <bool kLargest>
 __device__ __forceinline__ void warp_best(float& v, int& j) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     const float ov = __shfl_xor_sync(0xffffffffu, v, o);
     const int oj = __shfl_xor_sync(0xffffffffu, j, o);
-    const bool take = (oj != INT_MAX) &&
-                      (j == INT_MAX || (kLargest ? ov > v : ov < v) || (ov == v && oj < j));
-    if (take) {
+    if (beats<kLargest>(ov, oj, v, j)) {
       v = ov;
       j = oj;
     }
   }
 }
 
+// CTA-wide best (value, index) of every thread's candidate; the same result
+// in every thread.  Uses red_v / red_j [kRsWarps] and two barriers.
+template <bool kLargest>
+__device__ __forceinline__ void cta_best(float& v, int& j, float* red_v, int* red_j, int warp,
+                                         int lane) {
+  warp_best<kLargest>(v, j);
+  if (lane == 0) {
+    red_v[warp] = v;
+    red_j[warp] = j;
+  }
+  __syncthreads();
+  v = red_v[0];
+  j = red_j[0];
+#pragma unroll
+  for (int w = 1; w < kRsWarps; ++w)
+    if (beats<kLargest>(red_v[w], red_j[w], v, j)) {
+      v = red_v[w];
+      j = red_j[w];
+    }
+  __syncthreads();
+}
+
+// CTA-wide sum (fixed order: lanes by a shuffle tree, then warps 0..3).
+__device__ __forceinline__ float cta_add(float v, float* red, int warp, int lane) {
+  v = warp_add(v);
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float s = red[0];
+#pragma unroll
+  for (int w = 1; w < kRsWarps; ++w) s += red[w];
+  __syncthreads();
+  return s;
+}
+
 // out[j] = sum_d x[d] * mt[d][j] for every j < nb (d ascending, float32
-// FMA): lane l takes blocks l, l + 32, l + 64, l + 96 of each group of 128 at
-// once, four independent chains with their loads in flight together.  Loads
-// past nb stay inside the padded row (index clamped to nb_pad - 1) and are
-// not stored.
+// FMA): thread t takes blocks t, t + 128, t + 256, t + 384 of each group of
+// 512 at once, four independent chains.  Loads past nb stay inside the padded
+// row (index clamped to nb_pad - 1) and are not stored.
 __device__ __forceinline__ void dots4(const float* x, const float* __restrict__ mt, int nb_pad,
-                                      int nb, float* out, int lane) {
-  for (int j0 = lane; j0 < nb; j0 += 128) {
+                                      int nb, float* out, int tid) {
+  for (int j0 = tid; j0 < nb; j0 += 4 * kRsThreads) {
     int jj[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) jj[u] = min(j0 + 32 * u, nb_pad - 1);
+    for (int u = 0; u < 4; ++u) jj[u] = min(j0 + kRsThreads * u, nb_pad - 1);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 4
     for (int d = 0; d < kHeadDim; ++d) {
@@ -97,58 +138,65 @@ __device__ __forceinline__ void dots4(const float* x, const float* __restrict__ 
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u)
-      if (j0 + 32 * u < nb) out[j0 + 32 * u] = acc[u];
+      if (j0 + kRsThreads * u < nb) out[j0 + kRsThreads * u] = acc[u];
   }
 }
 
-__global__ void __launch_bounds__(32 * kRsMaxWarps) restore_kernel(const RestoreArgs a) {
+__global__ void __launch_bounds__(kRsThreads) restore_kernel(const RestoreArgs a) {
   extern __shared__ __align__(16) float rsm[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (blockDim.x >> 5) + warp;
-  if (row >= a.heads * a.nb) return;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int row = blockIdx.x;
   const int nb = a.nb, rs = a.row_stride;
   const int words = (nb + 31) >> 5;
-  // This warp's shared memory: p, the drift score / <T, Vbar_j>, |Vbar_j|^2
-  // (one row each), T, the candidates' contributions, their indices, the
-  // kept bitmap, the top-k scratch and the initial kept list.
-  float* p = rsm + (size_t)warp * a.warp_floats;
+  // Shared memory: p, the drift score / <T, Vbar_j>, |Vbar_j|^2, the initial
+  // kept list (one row each), T, the candidates' contributions, their
+  // indices, the kept bitmap, the top-k scratch and reduction slots.
+  float* p = rsm;
   float* dot = p + rs;
   float* vn2 = dot + rs;
-  float* T = vn2 + rs;                                         // [64]
-  float* cbv = T + 64;                                         // [kRsMaxCand][64]
-  float* cav = cbv + kRsMaxCand * 64;                          // [kRsMaxCand][64]
-  int* cb = reinterpret_cast<int*>(cav + kRsMaxCand * 64);     // [kRsMaxCand]
-  int* ca = cb + kRsMaxCand;                                   // [kRsMaxCand]
-  uint32_t* kept = reinterpret_cast<uint32_t*>(ca + kRsMaxCand);   // [128]
-  uint32_t* scratch = kept + 128;                              // [kWarpScratchStride]
-  int32_t* list = reinterpret_cast<int32_t*>(scratch + kWarpScratchStride);   // [rs]
+  int32_t* list = reinterpret_cast<int32_t*>(vn2 + rs);                 // [rs]
+  float* T = reinterpret_cast<float*>(list + rs);                      // [64]
+  float* cbv = T + 64;                                                 // [kRsMaxCand][64]
+  float* cav = cbv + kRsMaxCand * 64;                                  // [kRsMaxCand][64]
+  int* cb = reinterpret_cast<int*>(cav + kRsMaxCand * 64);             // [kRsMaxCand]
+  int* ca = cb + kRsMaxCand;                                           // [kRsMaxCand]
+  uint32_t* kept = reinterpret_cast<uint32_t*>(ca + kRsMaxCand);       // [128]
+  float* ored = reinterpret_cast<float*>(kept + 128);                  // [kRsWarps][64]
+  float* red_v = ored + kRsWarps * 64;                                 // [kRsWarps]
+  int* red_j = reinterpret_cast<int*>(red_v + kRsWarps);               // [kRsWarps]
+  uint32_t* scratch = reinterpret_cast<uint32_t*>(red_j + kRsWarps);   // [kWarpScratchStride]
 
   const int h = row / nb, i = row - h * nb;
   const float* kt = a.kbar_t + (size_t)h * kHeadDim * a.nb_pad;
   const float* vt = a.vbar_t + (size_t)h * kHeadDim * a.nb_pad;
   const float* qrow = a.qbar + ((size_t)h * nb + i) * kHeadDim;
-  if (lane < 16) reinterpret_cast<float4*>(T)[lane] = reinterpret_cast<const float4*>(qrow)[lane];
-  __syncwarp();
+  if (tid < 16) reinterpret_cast<float4*>(T)[tid] = reinterpret_cast<const float4*>(qrow)[tid];
+  for (int w = tid; w < 128; w += kRsThreads) kept[w] = 0u;
+  __syncthreads();
 
   // Pooled logits (d ascending, float32 FMA, exact 1/8) and probabilities.
-  dots4(T, kt, a.nb_pad, nb, p, lane);
+  dots4(T, kt, a.nb_pad, nb, p, tid);
   float m = -INFINITY;
-  for (int j = lane; j < nb; j += 32) {
+  for (int j = tid; j < nb; j += kRsThreads) {
     const float s = p[j] * 0.125f;
     p[j] = s;
     m = fmaxf(m, s);
   }
   m = warp_max(m);
+  if (lane == 0) red_v[warp] = m;
+  __syncthreads();
+  m = fmaxf(fmaxf(red_v[0], red_v[1]), fmaxf(red_v[2], red_v[3]));
+  __syncthreads();
   float z = 0.f;
-  for (int j = lane; j < nb; j += 32) z += expf(p[j] - m);
-  z = warp_add(z);
+  for (int j = tid; j < nb; j += kRsThreads) z += expf(p[j] - m);
+  z = cta_add(z, red_v, warp, lane);
   const float inv_z = 1.0f / z;
   // p_j, |Vbar_j|^2, the drift score p_j |Vbar_j| and the pooled output
-  // O = sum_j c_j, accumulated per lane over its blocks and reduced (d by d).
+  // O = sum_j c_j, accumulated per thread over its blocks and reduced.
   float o[kHeadDim];
 #pragma unroll
   for (int d = 0; d < kHeadDim; ++d) o[d] = 0.f;
-  for (int j = lane; j < nb; j += 32) {
+  for (int j = tid; j < nb; j += kRsThreads) {
     const float pj = expf(p[j] - m) * inv_z;
     float vv = 0.f;
 #pragma unroll
@@ -162,37 +210,42 @@ __global__ void __launch_bounds__(32 * kRsMaxWarps) restore_kernel(const Restore
     dot[j] = pj * sqrtf(vv);
   }
 #pragma unroll
-  for (int d = 0; d < kHeadDim; ++d) o[d] = warp_add(o[d]);
-  __syncwarp();
-  // Initial kept set: the budget largest drift scores, ties to the lower index.
-  warp_topk_row_binned(dot, nb, a.budget, scratch, list, lane);
-  __syncwarp();
-  for (int w = lane; w < 128; w += 32) kept[w] = 0u;
-  __syncwarp();
-  for (int r = lane; r < a.budget; r += 32) atomicOr(&kept[list[r] >> 5], 1u << (list[r] & 31));
-  __syncwarp();
-  // T = O - sum over the kept blocks of c_j (lane l holds d = l and l + 32).
-  float t0 = 0.f, t1 = 0.f;
-#pragma unroll
   for (int d = 0; d < kHeadDim; ++d) {
-    if (d == lane) t0 = o[d];
-    if (d == lane + 32) t1 = o[d];
+    const float od = warp_add(o[d]);
+    if (lane == 0) ored[warp * 64 + d] = od;
   }
-  for (int r = 0; r < a.budget; ++r) {
-    const int j = list[r];
-    t0 = fmaf(-p[j], vt[(size_t)lane * a.nb_pad + j], t0);
-    t1 = fmaf(-p[j], vt[(size_t)(lane + 32) * a.nb_pad + j], t1);
+  __syncthreads();
+  // Initial kept set: the budget largest drift scores, ties to the lower index.
+  if (warp == 0) warp_topk_row_binned(dot, nb, a.budget, scratch, list, lane);
+  __syncthreads();
+  for (int r = tid; r < a.budget; r += kRsThreads)
+    atomicOr(&kept[list[r] >> 5], 1u << (list[r] & 31));
+  // T = O - sum over the kept blocks of c_j: thread (d, half) sums half of the
+  // kept list for dimension d.
+  {
+    const int d = tid & 63, half = tid >> 6;
+    float acc = 0.f;
+    for (int r = half; r < a.budget; r += 2) {
+      const int j = list[r];
+      acc = fmaf(p[j], vt[(size_t)d * a.nb_pad + j], acc);
+    }
+    cbv[half * 64 + d] = acc;   // scratch use of the candidate area
   }
-  float jcur2 = warp_add(t0 * t0 + t1 * t1);
+  __syncthreads();
+  if (tid < 64)
+    T[tid] = ((ored[tid] + ored[64 + tid]) + (ored[128 + tid] + ored[192 + tid])) -
+             (cbv[tid] + cbv[64 + tid]);
+  __syncthreads();
+  float jcur2 = 0.f;
+  {
+    const float t = tid < 64 ? T[tid] : 0.f;
+    jcur2 = cta_add(t * t, red_v, warp, lane);
+  }
   const float j_init = sqrtf(jcur2);
 
   for (int round = 0; round < a.rounds; ++round) {
-    __syncwarp();
-    T[lane] = t0;
-    T[lane + 32] = t1;
-    __syncwarp();
-    dots4(T, vt, a.nb_pad, nb, dot, lane);
-    __syncwarp();
+    dots4(T, vt, a.nb_pad, nb, dot, tid);
+    __syncthreads();
     // Candidates: the dropped blocks of largest gain 2 <T, c_b> - |c_b|^2 and
     // the kept blocks of smallest cost 2 <T, c_a> + |c_a|^2.
     int nbc = 0, nac = 0;
@@ -202,7 +255,7 @@ __global__ void __launch_bounds__(32 * kRsMaxWarps) restore_kernel(const Restore
       for (int t = 0; t < a.cand; ++t) {
         float bv = 0.f;
         int bj = INT_MAX;
-        for (int j = lane; j < nb; j += 32) {
+        for (int j = tid; j < nb; j += kRsThreads) {
           const bool in_k = (kept[j >> 5] >> (j & 31)) & 1u;
           if (side == 0 ? in_k : !in_k) continue;
           bool taken = false;
@@ -212,36 +265,35 @@ __global__ void __launch_bounds__(32 * kRsMaxWarps) restore_kernel(const Restore
           const float c2 = pj * pj * vn2[j];
           const float lin = 2.0f * pj * dot[j];
           const float val = side == 0 ? lin - c2 : lin + c2;
-          if (bj == INT_MAX || (side == 0 ? val > bv : val < bv)) {
+          if (side == 0 ? beats<true>(val, j, bv, bj) : beats<false>(val, j, bv, bj)) {
             bv = val;
             bj = j;
           }
         }
-        if (side == 0) warp_best<true>(bv, bj); else warp_best<false>(bv, bj);
+        if (side == 0) cta_best<true>(bv, bj, red_v, red_j, warp, lane);
+        else cta_best<false>(bv, bj, red_v, red_j, warp, lane);
         if (bj == INT_MAX) break;
-        if (lane == 0) {
+        if (tid == 0) {
           if (side == 0) cb[t] = bj; else ca[t] = bj;
         }
-        __syncwarp();
+        __syncthreads();
         if (side == 0) nbc = t + 1; else nac = t + 1;
       }
     }
     if (nbc == 0 || nac == 0) break;
-    for (int u = 0; u < nbc; ++u) {
-      const int j = cb[u];
-      cbv[u * 64 + lane] = p[j] * vt[(size_t)lane * a.nb_pad + j];
-      cbv[u * 64 + lane + 32] = p[j] * vt[(size_t)(lane + 32) * a.nb_pad + j];
+    for (int e = tid; e < nbc * 64; e += kRsThreads) {
+      const int u = e >> 6, d = e & 63;
+      cbv[e] = p[cb[u]] * vt[(size_t)d * a.nb_pad + cb[u]];
     }
-    for (int u = 0; u < nac; ++u) {
-      const int j = ca[u];
-      cav[u * 64 + lane] = p[j] * vt[(size_t)lane * a.nb_pad + j];
-      cav[u * 64 + lane + 32] = p[j] * vt[(size_t)(lane + 32) * a.nb_pad + j];
+    for (int e = tid; e < nac * 64; e += kRsThreads) {
+      const int u = e >> 6, d = e & 63;
+      cav[e] = p[ca[u]] * vt[(size_t)d * a.nb_pad + ca[u]];
     }
-    __syncwarp();
+    __syncthreads();
     // The pair of smallest |T - c_b + c_a|^2 (ties: lower b, then lower a).
     float best = 0.f;
     int best_code = INT_MAX;
-    for (int e = lane; e < nbc * nac; e += 32) {
+    for (int e = tid; e < nbc * nac; e += kRsThreads) {
       const int ub = e / nac, ua = e - ub * nac;
       float s = 0.f;
 #pragma unroll 8
@@ -250,51 +302,52 @@ __global__ void __launch_bounds__(32 * kRsMaxWarps) restore_kernel(const Restore
         s = fmaf(x, x, s);
       }
       const int code = cb[ub] * nb + ca[ua];
-      if (best_code == INT_MAX || s < best || (s == best && code < best_code)) {
+      if (beats<false>(s, code, best, best_code)) {
         best = s;
         best_code = code;
       }
     }
-    warp_best<false>(best, best_code);
+    cta_best<false>(best, best_code, red_v, red_j, warp, lane);
     if (!(best < jcur2)) break;
     const int b = best_code / nb, aa = best_code - b * nb;
-    __syncwarp();
-    if (lane == 0) {
+    if (tid == 0) {
       kept[aa >> 5] &= ~(1u << (aa & 31));
       kept[b >> 5] |= 1u << (b & 31);
     }
-    __syncwarp();
-    t0 = t0 - p[b] * vt[(size_t)lane * a.nb_pad + b] + p[aa] * vt[(size_t)lane * a.nb_pad + aa];
-    t1 = t1 - p[b] * vt[(size_t)(lane + 32) * a.nb_pad + b] +
-         p[aa] * vt[(size_t)(lane + 32) * a.nb_pad + aa];
+    if (tid < 64)
+      T[tid] = T[tid] - p[b] * vt[(size_t)tid * a.nb_pad + b] +
+               p[aa] * vt[(size_t)tid * a.nb_pad + aa];
+    __syncthreads();
     jcur2 = best;
   }
-  // The kept blocks in ascending order.
-  int32_t* out = a.idx + ((size_t)h * nb + i) * a.budget;
-  int pos = 0;
-  for (int w0 = 0; w0 < words; w0 += 32) {
-    const int w = w0 + lane;
-    const uint32_t m32 = w < words ? kept[w] : 0u;
-    const int cnt = __popc(m32);
-    int incl = cnt;
+  // The kept blocks in ascending order (warp 0).
+  if (warp == 0) {
+    int32_t* out = a.idx + ((size_t)h * nb + i) * a.budget;
+    int pos = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+      const int w = w0 + lane;
+      const uint32_t m32 = w < words ? kept[w] : 0u;
+      const int cnt = __popc(m32);
+      int incl = cnt;
 #pragma unroll
-    for (int o2 = 1; o2 < 32; o2 <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, incl, o2);
-      if (lane >= o2) incl += y;
+      for (int o2 = 1; o2 < 32; o2 <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o2);
+        if (lane >= o2) incl += y;
+      }
+      int at = pos + incl - cnt;
+      uint32_t mm = m32;
+      while (mm) {
+        const int bit = __ffs(mm) - 1;
+        mm &= mm - 1u;
+        if (at < a.budget) out[at] = 32 * w + bit;
+        ++at;
+      }
+      pos += __shfl_sync(0xffffffffu, incl, 31);
     }
-    int at = pos + incl - cnt;
-    uint32_t mm = m32;
-    while (mm) {
-      const int bit = __ffs(mm) - 1;
-      mm &= mm - 1u;
-      if (at < a.budget) out[at] = 32 * w + bit;
-      ++at;
+    if (lane == 0) {
+      if (a.j_init) a.j_init[(size_t)h * nb + i] = j_init;
+      if (a.j_final) a.j_final[(size_t)h * nb + i] = sqrtf(jcur2);
     }
-    pos += __shfl_sync(0xffffffffu, incl, 31);
-  }
-  if (lane == 0) {
-    if (a.j_init) a.j_init[(size_t)h * nb + i] = j_init;
-    if (a.j_final) a.j_final[(size_t)h * nb + i] = sqrtf(jcur2);
   }
 }
 
@@ -335,20 +388,14 @@ ress_status launch_restore(const Geometry& g, const void* q, const void* k, cons
   a.rounds = rounds;
   a.cand = cand;
   a.row_stride = (g.nb + 3) & ~3;
-  a.warp_floats = 4 * a.row_stride + 64 + 2 * kRsMaxCand * 64 + 2 * kRsMaxCand + 128 +
-                  kWarpScratchStride;
-  a.warp_floats = (a.warp_floats + 3) & ~3;
-  // As many rows per CTA as fit (nb = 4,096 leaves room for two).
-  const size_t per_warp = sizeof(float) * (size_t)a.warp_floats;
-  int warps = (int)((227 * 1024) / per_warp);
-  if (warps > kRsMaxWarps) warps = kRsMaxWarps;
-  if (warps < 1) return RESS_ERR_UNSUPPORTED;
-  const size_t smem = per_warp * warps;
+  const size_t floats = 4 * (size_t)a.row_stride + 64 + 2 * kRsMaxCand * 64 + 2 * kRsMaxCand +
+                        128 + kRsWarps * 64 + 2 * kRsWarps + kWarpScratchStride;
+  const size_t smem = sizeof(float) * floats;
+  if (smem > 227 * 1024) return RESS_ERR_UNSUPPORTED;
   if (ress_status s = record_cuda(cudaFuncSetAttribute(
           restore_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
     return s;
-  const int rows = g.heads * g.nb;
-  restore_kernel<<<(rows + warps - 1) / warps, 32 * warps, smem, st>>>(a);
+  restore_kernel<<<g.heads * g.nb, kRsThreads, smem, st>>>(a);
   return record_cuda(cudaGetLastError());
 }
 
