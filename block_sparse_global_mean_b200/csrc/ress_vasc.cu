@@ -31,7 +31,7 @@ namespace ress {
 
 namespace {
 
-constexpr int kPrepThreads = 256;
+constexpr int kPrepThreads = 1024;   // one or two pairs per thread at nb = 2,200
 
 struct VascPrepArgs {
   const float* vbar_t;   // [H][64][nb_pad] (null when the contrast is off)
@@ -56,11 +56,18 @@ __global__ void __launch_bounds__(kPrepThreads) vasc_prep_kernel(const VascPrepA
       r = 0.f;
       if (2 * p + 1 < a.nb) {
         const float* vt = a.vbar_t + (size_t)h * kHeadDim * a.nb_pad + 2 * p;
-        float s = 0.f;
-        for (int d = 0; d < kHeadDim; ++d) {
-          const float x = vt[(size_t)d * a.nb_pad] - vt[(size_t)d * a.nb_pad + 1];
-          s = fmaf(x, x, s);
+        // Four partial sums over d (independent loads in flight), added in a
+        // fixed order.
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+        for (int d = 0; d < kHeadDim; d += 4) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float x = vt[(size_t)(d + u) * a.nb_pad] - vt[(size_t)(d + u) * a.nb_pad + 1];
+            s4[u] = fmaf(x, x, s4[u]);
+          }
         }
+        const float s = (s4[0] + s4[1]) + (s4[2] + s4[3]);
         r = sqrtf(s * (1.0f / kHeadDim));   // 1/64 is exact
       }
     }
