@@ -102,18 +102,24 @@ size_t attn_smem_bytes(int nb) {
          sizeof(uint32_t) * (2 * (size_t)words_for(nb) + (size_t)nb);
 }
 
+// Entry of the sorted list: bits 0..13 the key block (nb <= 16,383), bits
+// 30..31 which row halves use it (bit 0: rows 0..63, bit 1: rows 64..127);
+// with a layout, bits 14..20 the valid (non-padding) tokens of the block's
+// first 64 and bits 21..27 of its second 64 (128-token blocks).
+constexpr uint32_t kEntryBlock = 0x3FFFu;
+constexpr int kMaxAttnBlocks = 16383;
+
 // Chunk c of the sorted entry list -> token starts of its two 64-key
-// sub-blocks and, per sub-block, which row halves use it (bit 0: rows 0..63,
-// bit 1: rows 64..127).
+// sub-blocks and, per sub-block, which row halves use it.
 __device__ __forceinline__ void chunk_info(const uint32_t* list, int n_entries, int block, int c,
                                            int& t0, int& t1, uint32_t& m0, uint32_t& m1) {
   if (block == 64) {
     const uint32_t e0 = list[2 * c];
-    t0 = (int)(e0 & 0x3FFFFFFFu) * 64;
+    t0 = (int)(e0 & kEntryBlock) * 64;
     m0 = e0 >> 30;
     if (2 * c + 1 < n_entries) {
       const uint32_t e1 = list[2 * c + 1];
-      t1 = (int)(e1 & 0x3FFFFFFFu) * 64;
+      t1 = (int)(e1 & kEntryBlock) * 64;
       m1 = e1 >> 30;
     } else {  // odd count: repeat a valid sub-block, masked for every row
       t1 = t0;
@@ -121,9 +127,22 @@ __device__ __forceinline__ void chunk_info(const uint32_t* list, int n_entries, 
     }
   } else {
     const uint32_t e0 = list[c];
-    t0 = (int)(e0 & 0x3FFFFFFFu) * 128;
+    t0 = (int)(e0 & kEntryBlock) * 128;
     t1 = t0 + 64;
     m0 = m1 = 3u;
+  }
+}
+
+// Valid-token prefixes of chunk c's two sub-blocks (layouts only).
+__device__ __forceinline__ void chunk_valid(const uint32_t* list, int n_entries, int block, int c,
+                                            int& vk0, int& vk1) {
+  if (block == 64) {
+    vk0 = (int)((list[2 * c] >> 14) & 0x7Fu);
+    vk1 = (2 * c + 1 < n_entries) ? (int)((list[2 * c + 1] >> 14) & 0x7Fu) : vk0;
+  } else {
+    const uint32_t e0 = list[c];
+    vk0 = (int)((e0 >> 14) & 0x7Fu);
+    vk1 = (int)((e0 >> 21) & 0x7Fu);
   }
 }
 
@@ -287,7 +306,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int bit = __ffs(u) - 1;
         u &= u - 1u;
         const uint32_t mem = ((a >> bit) & 1u) | (((b >> bit) & 1u) << 1);
-        list[pos++] = (uint32_t)(w * 32 + bit) | (mem << 30);
+        uint32_t e = (uint32_t)(w * 32 + bit) | (mem << 30);
+        if (kLayout) {   // valid prefixes, once per block instead of once per chunk and thread
+          const int tb = (w * 32 + bit) * p.block;
+          e |= (uint32_t)layout_valid(p.lay_t, p.lay_r, tb, 64) << 14;
+          if (p.block == 128) e |= (uint32_t)layout_valid(p.lay_t, p.lay_r, tb + 64, 64) << 21;
+        }
+        list[pos++] = e;
       }
       base += __shfl_sync(0xffffffffu, incl, 31);
     }
@@ -435,8 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t m0, m1;
       chunk_info(list, n_entries, p.block, c, t0, t1, m0, m1);
       // Valid (non-padding) prefix of each 64-key sub-block.
-      const int vk0 = kLayout ? layout_valid(p.lay_t, p.lay_r, t0, 64) : 64;
-      const int vk1 = kLayout ? layout_valid(p.lay_t, p.lay_r, t1, 64) : 64;
+      int vk0 = 64, vk1 = 64;
+      if (kLayout) chunk_valid(list, n_entries, p.block, c, vk0, vk1);
       const bool use0 = ((m0 >> half) & 1u) && vk0 > 0;
       const bool use1 = ((m1 >> half) & 1u) && vk1 > 0;
       if (!use0 && !use1) {
@@ -680,7 +705,8 @@ ress_status launch_attn_rows(const Geometry& g, const void* q, int64_t nq, bool 
   p.out = out;
   p.lse = lse;
   const size_t smem = attn_smem_bytes(g.nb);
-  if (smem > 227 * 1024) return RESS_ERR_UNSUPPORTED;   // kept-block lists no longer fit
+  if (smem > 227 * 1024 || g.nb > kMaxAttnBlocks)
+    return RESS_ERR_UNSUPPORTED;   // kept-block lists no longer fit
   const dim3 grid((unsigned)(g.heads * p.tiles_per_head));
   // The plain path is compiled without any of the layout's checks.
   const bool lay = g.lay_t != 0 || dense;

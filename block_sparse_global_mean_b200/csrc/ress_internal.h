@@ -34,6 +34,12 @@ __host__ __device__ inline int layout_valid(int lay_t, int lay_r, long long t0, 
   const int v = lay_r - (int)(t0 % lay_t);
   return v < 0 ? 0 : (v > len ? len : v);
 }
+// The same for a token index below 2^31 (a 32-bit remainder).
+__host__ __device__ inline int layout_valid(int lay_t, int lay_r, int t0, int len) {
+  if (lay_t == 0) return len;
+  const int v = lay_r - (int)((unsigned)t0 % (unsigned)lay_t);
+  return v < 0 ? 0 : (v > len ? len : v);
+}
 
 constexpr int kHeadDim = 64;
 constexpr int kMaxHeads = 64;
