@@ -186,3 +186,30 @@ def test_vasc_views100_sampled_rows(ress_gpu, wcache):
     rows = set(sample_rows(w.heads, w.n_blocks, count=96))
     _check_layer(q, k, v, w.block, budgets, w.budget, mem_in, idx, dem, ser,
                  mem.cpu().numpy().astype(np.float64), rows=rows)
+
+
+def test_vasc_64_heads_with_budgets_from_one_to_capacity(ress_gpu):
+    # The head maximum: every c_h from 1 to the capacity (32 blocks, capacity 16).
+    g = torch.Generator().manual_seed(64)
+    n, h = 32 * 64, 64
+    q, k, v = (torch.randn(n, h, 64, generator=g).to("cuda", torch.bfloat16) for _ in range(3))
+    budgets = [1 + (hh % 16) for hh in range(h)]
+    mem = (torch.rand((h, 16), generator=g) * 0.3).to("cuda")
+    mem_in = mem.cpu().numpy().astype(np.float64)
+    idx, dem, ser = _run(ress_gpu, q, k, v, budgets, 64, 16, mem)
+    _check_layer(q, k, v, 64, budgets, 16, mem_in, idx, dem, ser, mem.cpu().numpy().astype(np.float64))
+
+
+def test_vasc_reset_ignores_the_memory_passed_in(ress_gpu):
+    # reset = 1 starts an inference: a non-zero memory gives exactly what a
+    # zeroed one gives, and is overwritten by the settled state.
+    w = workloads.WORKLOADS["vggt8"]
+    q, k, v = _layer_inputs(w, 0)
+    pairs = ress_gpu.vasc_pairs(w.n_blocks)
+    a = torch.full((w.heads, pairs), 7.0, device="cuda")
+    b = torch.zeros((w.heads, pairs), device="cuda")
+    ra = _run(ress_gpu, q, k, v, [50] * w.heads, w.block, 50, a, reset=True)
+    rb = _run(ress_gpu, q, k, v, [50] * w.heads, w.block, 50, b, reset=False)
+    for x, y in zip(ra, rb):
+        assert np.array_equal(x, y)
+    assert torch.equal(a, b)
