@@ -133,3 +133,58 @@ def test_head_slice_rejects_uneven_splits():
     assert bench.head_slice(16, 4, 3) == (12, 16)
     with pytest.raises(ValueError):
         bench.head_slice(16, 3, 0)
+
+
+def _vasc_head_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import numpy as np
+
+    import bench
+    import oracle
+    from block_sparse_global_mean_b200 import workloads
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        w = workloads.scaled(workloads.WORKLOADS["vggt8"], 1, name="split")   # 22 blocks, H=16
+        budgets = [3 + (h % 7) for h in range(w.heads)]
+        h0, h1 = bench.head_slice(w.heads, world, rank)
+        mem = None
+        mine = []
+        for layer in range(2):
+            full = workloads.generate(w, seed=w.seed + 1000 * (layer + 1))
+            qs, ks, vs = (t.double().numpy() for t in bench.shard_heads(full, h0, h1))
+            idx, mem, _ = oracle.select_blocks_vasc(qs, ks, vs, w.block, budgets[h0:h1], 9, mem)
+            mine.append((idx, mem))
+        parts = [None] * world
+        dist.all_gather_object(parts, (h0, h1, mine))
+        if rank == 0:
+            ok = True
+            ref_mem = None
+            for layer in range(2):
+                full = workloads.generate(w, seed=w.seed + 1000 * (layer + 1))
+                qf, kf, vf = (t.double().numpy() for t in full)
+                ref_idx, ref_mem, _ = oracle.select_blocks_vasc(qf, kf, vf, w.block, budgets, 9,
+                                                                ref_mem)
+                for a, b, rmine in parts:
+                    ok &= np.array_equal(rmine[layer][0], ref_idx[a:b])
+                    ok &= np.allclose(rmine[layer][1], ref_mem[a:b], rtol=0, atol=1e-15)
+            q.put(ok)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_vasc_head_split_over_two_gloo_ranks_equals_the_unsharded_layers():
+    """The VASC layer shards by head: each rank keeps its heads' memory, and
+    two layers on two ranks give the kept sets and memory of the unsharded
+    run (the memory copy is normalised per head, budgets are per head)."""
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_vasc_head_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    ok = q.get(timeout=300)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert ok
