@@ -142,6 +142,67 @@ __device__ __forceinline__ void dots4(const float* x, const float* __restrict__ 
   }
 }
 
+// The `a.cand` best blocks of one side into out[] (kLargest: the dropped
+// blocks of largest gain; else the kept blocks of smallest cost), ties to the
+// lower index; their number goes to n.  Returns whether any was found.
+template <bool kLargest>
+__device__ __forceinline__ bool side_candidates(const RestoreArgs& a, const uint32_t* kept,
+                                                const float* p, const float* vn2,
+                                                const float* dot, int* out, float* red_v,
+                                                int* red_j, int tid, int warp, int lane, int nb,
+                                                int& n) {
+  float v[kRsMaxCand];
+  int jx[kRsMaxCand];
+#pragma unroll
+  for (int u = 0; u < kRsMaxCand; ++u) {
+    v[u] = 0.f;
+    jx[u] = INT_MAX;
+  }
+  for (int j = tid; j < nb; j += kRsThreads) {
+    const bool in_k = (kept[j >> 5] >> (j & 31)) & 1u;
+    if (kLargest ? in_k : !in_k) continue;
+    const float pj = p[j];
+    const float c2 = pj * pj * vn2[j];
+    const float lin = 2.0f * pj * dot[j];
+    float cv = kLargest ? lin - c2 : lin + c2;
+    int cj = j;
+    if (!beats<kLargest>(cv, cj, v[kRsMaxCand - 1], jx[kRsMaxCand - 1])) continue;
+    // Insert: the carried entry swaps with every slot it beats.
+#pragma unroll
+    for (int u = 0; u < kRsMaxCand; ++u) {
+      if (beats<kLargest>(cv, cj, v[u], jx[u])) {
+        const float tv = v[u];
+        const int tj = jx[u];
+        v[u] = cv;
+        jx[u] = cj;
+        cv = tv;
+        cj = tj;
+      }
+    }
+  }
+  n = 0;
+#pragma unroll 1
+  for (int t = 0; t < a.cand; ++t) {
+    float bv = v[0];
+    int bj = jx[0];
+    cta_best<kLargest>(bv, bj, red_v, red_j, warp, lane);
+    if (bj == INT_MAX) break;
+    if (jx[0] == bj) {   // this thread's head won: pop it
+#pragma unroll
+      for (int u = 0; u + 1 < kRsMaxCand; ++u) {
+        v[u] = v[u + 1];
+        jx[u] = jx[u + 1];
+      }
+      v[kRsMaxCand - 1] = 0.f;
+      jx[kRsMaxCand - 1] = INT_MAX;
+    }
+    if (tid == 0) out[t] = bj;
+    n = t + 1;
+  }
+  __syncthreads();
+  return n > 0;
+}
+
 __global__ void __launch_bounds__(kRsThreads) restore_kernel(const RestoreArgs a) {
   extern __shared__ __align__(16) float rsm[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -247,39 +308,13 @@ __global__ void __launch_bounds__(kRsThreads) restore_kernel(const RestoreArgs a
     dots4(T, vt, a.nb_pad, nb, dot, tid);
     __syncthreads();
     // Candidates: the dropped blocks of largest gain 2 <T, c_b> - |c_b|^2 and
-    // the kept blocks of smallest cost 2 <T, c_a> + |c_a|^2.
-    int nbc = 0, nac = 0;
-#pragma unroll 1
-    for (int side = 0; side < 2; ++side) {
-#pragma unroll 1
-      for (int t = 0; t < a.cand; ++t) {
-        float bv = 0.f;
-        int bj = INT_MAX;
-        for (int j = tid; j < nb; j += kRsThreads) {
-          const bool in_k = (kept[j >> 5] >> (j & 31)) & 1u;
-          if (side == 0 ? in_k : !in_k) continue;
-          bool taken = false;
-          for (int u = 0; u < t; ++u) taken |= (side == 0 ? cb[u] : ca[u]) == j;
-          if (taken) continue;
-          const float pj = p[j];
-          const float c2 = pj * pj * vn2[j];
-          const float lin = 2.0f * pj * dot[j];
-          const float val = side == 0 ? lin - c2 : lin + c2;
-          if (side == 0 ? beats<true>(val, j, bv, bj) : beats<false>(val, j, bv, bj)) {
-            bv = val;
-            bj = j;
-          }
-        }
-        if (side == 0) cta_best<true>(bv, bj, red_v, red_j, warp, lane);
-        else cta_best<false>(bv, bj, red_v, red_j, warp, lane);
-        if (bj == INT_MAX) break;
-        if (tid == 0) {
-          if (side == 0) cb[t] = bj; else ca[t] = bj;
-        }
-        __syncthreads();
-        if (side == 0) nbc = t + 1; else nac = t + 1;
-      }
-    }
+    // the kept blocks of smallest cost 2 <T, c_a> + |c_a|^2 (ties to the
+    // lower index).  Each thread keeps its best kRsMaxCand of a side in
+    // registers in one pass over its blocks, then the CTA takes the best
+    // `cand` by repeatedly choosing among the threads' heads.
+    int nbc = 0, nac = 0;   // the same in every thread: every branch below is uniform
+    if (side_candidates<true>(a, kept, p, vn2, dot, cb, red_v, red_j, tid, warp, lane, nb, nbc))
+      side_candidates<false>(a, kept, p, vn2, dot, ca, red_v, red_j, tid, warp, lane, nb, nac);
     if (nbc == 0 || nac == 0) break;
     for (int e = tid; e < nbc * 64; e += kRsThreads) {
       const int u = e >> 6, d = e & 63;
