@@ -119,26 +119,34 @@ __device__ __forceinline__ float cta_add(float v, float* red, int warp, int lane
 }
 
 // out[j] = sum_d x[d] * mt[d][j] for every j < nb (d ascending, float32
-// FMA): thread t takes blocks t, t + 128, t + 256, t + 384 of each group of
-// 512 at once, four independent chains.  Loads past nb stay inside the padded
-// row (index clamped to nb_pad - 1) and are not stored.
+// FMA, one chain per j): thread t takes the four consecutive blocks 4t .. 4t+3
+// of each group of 512 with one 16-byte load per d and two packed FMAs.  The
+// rows of mt are nb_pad (a multiple of 256) floats, so the loads past nb stay
+// inside the row; those results are not stored.
 __device__ __forceinline__ void dots4(const float* x, const float* __restrict__ mt, int nb_pad,
                                       int nb, float* out, int tid) {
-  for (int j0 = tid; j0 < nb; j0 += 4 * kRsThreads) {
-    int jj[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) jj[u] = min(j0 + kRsThreads * u, nb_pad - 1);
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int j0 = 4 * tid; j0 < nb; j0 += 4 * kRsThreads) {
+    float2 a01 = make_float2(0.f, 0.f), a23 = make_float2(0.f, 0.f);
 #pragma unroll 4
-    for (int d = 0; d < kHeadDim; ++d) {
-      const float xd = x[d];
-      const float* row = mt + (size_t)d * nb_pad;
+    for (int d4 = 0; d4 < kHeadDim; d4 += 4) {
+      const float4 xv = *reinterpret_cast<const float4*>(x + d4);
+      const float xs[4] = {xv.x, xv.y, xv.z, xv.w};
 #pragma unroll
-      for (int u = 0; u < 4; ++u) acc[u] = fmaf(xd, row[jj[u]], acc[u]);
+      for (int u = 0; u < 4; ++u) {
+        const float4 m = *reinterpret_cast<const float4*>(mt + (size_t)(d4 + u) * nb_pad + j0);
+        const float2 xx = make_float2(xs[u], xs[u]);
+        a01 = ffma2(xx, make_float2(m.x, m.y), a01);
+        a23 = ffma2(xx, make_float2(m.z, m.w), a23);
+      }
     }
+    if (j0 + 3 < nb) {
+      *reinterpret_cast<float4*>(out + j0) = make_float4(a01.x, a01.y, a23.x, a23.y);
+    } else {
+      const float r[4] = {a01.x, a01.y, a23.x, a23.y};
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (j0 + kRsThreads * u < nb) out[j0 + kRsThreads * u] = acc[u];
+      for (int u = 0; u < 4; ++u)
+        if (j0 + u < nb) out[j0 + u] = r[u];
+    }
   }
 }
 
@@ -237,6 +245,7 @@ __global__ void __launch_bounds__(kRsThreads) restore_kernel(const RestoreArgs a
 
   // Pooled logits (d ascending, float32 FMA, exact 1/8) and probabilities.
   dots4(T, kt, a.nb_pad, nb, p, tid);
+  __syncthreads();   // the logits were written by other threads than read them below
   float m = -INFINITY;
   for (int j = tid; j < nb; j += kRsThreads) {
     const float s = p[j] * 0.125f;
