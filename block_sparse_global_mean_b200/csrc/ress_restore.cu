@@ -1,5 +1,5 @@
 // ReSS-style drift-based selection with iterative restoration, on pooled
-// contributions (one warp per (head, query block) row).
+// contributions (one CTA per (head, query block) row).
 //
 // For query block i of head h, with p_ij the pooled probabilities of stage 1
 // (softmax over all key blocks of Qbar_i . Kbar_j / sqrt(d)) and Vbar_j the
@@ -18,8 +18,9 @@
 // values, the per-round products with T) are split over all 128 threads, the
 // row's probabilities, drift scores, value norms and candidate contributions
 // live in shared memory, and the pooled keys and values (transposed,
-// [64][nb_pad] per head) are read from the workspace.  Sums across threads
-// follow a fixed order, so the result is deterministic.
+// [64][nb_pad] per head) are read from the workspace.  Each thread keeps its
+// best candidates of a side in registers and the CTA merges them.  Sums
+// across threads follow a fixed order, so the result is deterministic.
 //
 // Sources: ReSS (thelatestinai.com) Abstract and Fig. 1 (drift: the shift a
 // masked block leaves in the residual stream; the drift of a drop set depends
