@@ -57,6 +57,20 @@ def main():
     ld, lj = oracle.drift_layout_block(q, k, v, lidx[1, 3], ll, 1, 3, w.block, valid, special)
     fixture["layout_drift_h1_i3"] = ld.tolist()
     fixture["layout_J_h1_i3"] = lj
+    # Restoration-based selection (4 rounds, 8 candidates).
+    ridx, rj0, rj1 = oracle.select_blocks_restore(q, k, v, w.block, w.budget, 4, 8)
+    fixture["restore_idx"] = ridx.tolist()
+    fixture["restore_j_init"] = rj0.tolist()
+    fixture["restore_j_final"] = rj1.tolist()
+    # VASC: three layers (layer l drawn with seed + 1000 (l + 1)), budgets 3 and
+    # 5, rows of 6, the memory carried from layer to layer.
+    mem = None
+    for layer in range(3):
+        ql, kl, vl = (t.to(torch.float64).numpy()
+                      for t in workloads.generate(w, seed=w.seed + 1000 * (layer + 1)))
+        vidx, mem, _ = oracle.select_blocks_vasc(ql, kl, vl, w.block, [3, 5], 6, mem)
+        fixture[f"vasc_idx_layer{layer}"] = vidx.tolist()
+        fixture[f"vasc_memory_layer{layer}"] = mem.tolist()
     with open(os.path.join(HERE, "oracle_tiny.json"), "w") as f:
         json.dump(fixture, f, indent=1)
         f.write("\n")

@@ -49,3 +49,21 @@ def test_oracle_reproduces_recorded_cdf_and_layout_outputs():
     ld, lj = oracle.drift_layout_block(q, k, v, lidx[1, 3], ll, 1, 3, w.block, valid, special)
     np.testing.assert_allclose(ld, g["layout_drift_h1_i3"], rtol=1e-12, atol=1e-300)
     np.testing.assert_allclose(lj, g["layout_J_h1_i3"], rtol=1e-12)
+
+
+def test_oracle_reproduces_recorded_restore_and_vasc_outputs():
+    with open(os.path.join(HERE, "oracle_tiny.json")) as f:
+        g = json.load(f)
+    w = workloads.WORKLOADS["tiny"]
+    q, k, v = (t.to(torch.float64).numpy() for t in workloads.generate(w))
+    ridx, rj0, rj1 = oracle.select_blocks_restore(q, k, v, w.block, w.budget, 4, 8)
+    np.testing.assert_array_equal(ridx, np.array(g["restore_idx"]))
+    np.testing.assert_allclose(rj0, g["restore_j_init"], rtol=1e-12)
+    np.testing.assert_allclose(rj1, g["restore_j_final"], rtol=1e-12)
+    mem = None
+    for layer in range(3):
+        ql, kl, vl = (t.to(torch.float64).numpy()
+                      for t in workloads.generate(w, seed=w.seed + 1000 * (layer + 1)))
+        vidx, mem, _ = oracle.select_blocks_vasc(ql, kl, vl, w.block, [3, 5], 6, mem)
+        np.testing.assert_array_equal(vidx, np.array(g[f"vasc_idx_layer{layer}"]))
+        np.testing.assert_allclose(mem, g[f"vasc_memory_layer{layer}"], rtol=1e-12, atol=1e-15)
